@@ -1,0 +1,168 @@
+"""fp64 CPU oracle for exact top-k sparse decode attention.
+
+TEST INFRASTRUCTURE ONLY: the test suite, ``__graft_entry__.smoke()`` and the CPU-baseline leg
+of ``bench.py`` may use this package; the product library never does.  It is independent of
+the CUDA path: it imports nothing from ``sparse_attention_decode_sd_b200`` and shares no code
+with it.  The arithmetic lives in ``oracle.c`` (plain loops in double precision); this module
+only compiles it with gcc and marshals tensors.
+
+Functions (all inputs are CPU tensors; bf16 tensors are read as their raw 16-bit patterns):
+
+* ``scores(shape, q, K, page_table, lens, b, h)``  -> float64 [N_b]
+      s_i = q[b,h] . K[b, h/G, i]  (the QK^T term of SDPA, "Sparse Attention inference
+      survey" (xllm), sec. 1.1).
+* ``topk(shape, q, K, page_table, lens, k)``        -> int32 [B, Hq, k_max]
+      exact top-k per (b, h), ties to the lower position, ascending, -1 padded
+      ("Technische Zusammenfassung: Kontextsparsitaet bei der Inferenzzeit", sec. 2,
+      "Oracle Top-K").
+* ``attend(shape, q, K, V, page_table, lens, idx)`` -> float64 [B, Hq, d]
+      softmax(s/sqrt(d)) V over the listed rows only (SDPA restricted to the selected set;
+      "Inference-time context sparsity: illusion or opportunity?", Fig. 1(a) "Sparse").
+* ``dense(shape, q, K, V, page_table, lens)``       -> float64 [B, Hq, d]
+      the same over all N_b rows (Fig. 1(a) "Dense").
+
+Parity status: every function above is pinned by tests/test_oracle.py (closed forms, brute
+force, library SDPA, invariants); none is "parity unpinned".
+"""
+from __future__ import annotations
+
+import contextlib
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def compile_source(src: str, out: str) -> str:
+    """gcc -O2 with OpenMP: one C file to one shared library."""
+    tmp = out + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-Wall", "-Wextra",
+           "-o", tmp, src, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, out)
+    return out
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into liboracle.so next to it."""
+    if not force and os.path.exists(_LIB_PATH) and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC):
+        return _LIB_PATH
+    return compile_source(_SRC, _LIB_PATH)
+
+
+def _configure(lib):
+    P = ctypes.c_void_p
+    I = ctypes.c_int
+    lib.oracle_scores.argtypes = [I] * 7 + [P, P, P, P, I, I, P]
+    lib.oracle_topk.argtypes = [I] * 8 + [P, P, P, P, P, P]
+    lib.oracle_attend.argtypes = [I] * 8 + [P, P, P, P, P, P, P]
+    lib.oracle_dense.argtypes = [I] * 7 + [P, P, P, P, P, P]
+    for f in (lib.oracle_scores, lib.oracle_topk, lib.oracle_attend, lib.oracle_dense):
+        f.restype = ctypes.c_int
+    lib.oracle_num_threads.restype = ctypes.c_int
+    return lib
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            _lib = _configure(ctypes.CDLL(build()))
+    return _lib
+
+
+@contextlib.contextmanager
+def use_library(path: str):
+    """Route this module's functions through another build of oracle.c (the pin tests use it to
+    show that deliberately broken copies of the oracle fail them)."""
+    global _lib
+    prev = _load()
+    with _lock:
+        _lib = _configure(ctypes.CDLL(path))
+    try:
+        yield
+    finally:
+        with _lock:
+            _lib = prev
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def _u16(t: torch.Tensor) -> np.ndarray:
+    if t.dtype != torch.bfloat16:
+        raise TypeError(f"expected a bfloat16 tensor, got {t.dtype}")
+    return np.ascontiguousarray(t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16))
+
+
+def _i32(t) -> np.ndarray:
+    if isinstance(t, torch.Tensor):
+        t = t.detach().cpu().numpy()
+    return np.ascontiguousarray(np.asarray(t, dtype=np.int32))
+
+
+def _p(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _dims(shape: dict):
+    return (int(shape["B"]), int(shape["Hq"]), int(shape["Hkv"]), int(shape["d"]), int(shape["P"]),
+            int(shape["max_pages"]))
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise ValueError(f"oracle {what} rejected its arguments (code {rc})")
+
+
+def scores(shape: dict, q, K, page_table, lens, b: int, h: int) -> np.ndarray:
+    B, Hq, Hkv, d, P, max_pages = _dims(shape)
+    qa, Ka, pt, ln = _u16(q), _u16(K), _i32(page_table), _i32(lens)
+    num_pages = Ka.size // (P * Hkv * d)
+    out = np.zeros(max(int(ln[b]), 1), dtype=np.float64)
+    _check(_load().oracle_scores(B, Hq, Hkv, d, P, max_pages, num_pages, _p(qa), _p(Ka), _p(pt), _p(ln),
+                                 int(b), int(h), _p(out)), "scores")
+    return out[: int(ln[b])]
+
+
+def topk(shape: dict, q, K, page_table, lens, k, k_max: int | None = None) -> np.ndarray:
+    B, Hq, Hkv, d, P, max_pages = _dims(shape)
+    k_max = int(shape["k_max"] if k_max is None else k_max)
+    qa, Ka, pt, ln, ka = _u16(q), _u16(K), _i32(page_table), _i32(lens), _i32(k)
+    num_pages = Ka.size // (P * Hkv * d)
+    idx = np.full((B, Hq, max(k_max, 0)), -1, dtype=np.int32)
+    _check(_load().oracle_topk(B, Hq, Hkv, d, P, max_pages, num_pages, k_max, _p(qa), _p(Ka), _p(pt), _p(ln),
+                               _p(ka), _p(idx)), "topk")
+    return idx
+
+
+def attend(shape: dict, q, K, V, page_table, lens, idx) -> np.ndarray:
+    B, Hq, Hkv, d, P, max_pages = _dims(shape)
+    qa, Ka, Va, pt, ln = _u16(q), _u16(K), _u16(V), _i32(page_table), _i32(lens)
+    ix = _i32(idx)
+    k_max = ix.shape[-1]
+    num_pages = Ka.size // (P * Hkv * d)
+    out = np.zeros((B, Hq, d), dtype=np.float64)
+    _check(_load().oracle_attend(B, Hq, Hkv, d, P, max_pages, num_pages, k_max, _p(qa), _p(Ka), _p(Va), _p(pt),
+                                 _p(ln), _p(ix), _p(out)), "attend")
+    return out
+
+
+def dense(shape: dict, q, K, V, page_table, lens) -> np.ndarray:
+    B, Hq, Hkv, d, P, max_pages = _dims(shape)
+    qa, Ka, Va, pt, ln = _u16(q), _u16(K), _u16(V), _i32(page_table), _i32(lens)
+    num_pages = Ka.size // (P * Hkv * d)
+    out = np.zeros((B, Hq, d), dtype=np.float64)
+    _check(_load().oracle_dense(B, Hq, Hkv, d, P, max_pages, num_pages, _p(qa), _p(Ka), _p(Va), _p(pt), _p(ln),
+                                _p(out)), "dense")
+    return out

@@ -1,0 +1,266 @@
+/*
+ * oracle.c -- plain, slow, fp64 CPU restatement of exact top-k sparse decode attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or call this file;
+ * only the test suite, the smoke check and the benchmark's CPU-baseline leg do.  It shares
+ * no code, header, table or constant with the CUDA library and includes none of its files.
+ *
+ * What it computes (every step in double precision, no blocking, fusion or reordering):
+ *
+ *   score      s[b,h,i] = sum_j q[b,h,j] * K[b, h/G, i, j]              for 0 <= i < N_b
+ *              -- the QK^T term of scaled dot-product attention
+ *                 ("Sparse Attention inference survey" (xllm), sec. 1.1, the SDPA formula);
+ *                 the 1/sqrt(d) factor is monotone and so does not change which rows win.
+ *   select     S[b,h] = the k_b positions with the largest s, ties at the k-th score going to
+ *              the lower position -- exact top-k
+ *              ("Technische Zusammenfassung: Kontextsparsitaet bei der Inferenzzeit",
+ *               sec. 2 "Sparsitaetsmechanismen: Oracle Top-K"; "Inference-time context
+ *               sparsity: illusion or opportunity?", Fig. 1(a): the indexer keeps k rows).
+ *   attend     out[b,h] = sum_{i in S} softmax_S(s_i / sqrt(d)) V[b, h/G, i]
+ *              -- SDPA restricted to the selected rows, softmax renormalised over S only
+ *              (same SDPA formula; Fig. 1(a) "Sparse" mode reads only the k selected rows).
+ *   dense      attend with S = all N_b positions (Fig. 1(a) "Dense" mode).
+ *
+ * Data layout read here (the paged KV cache the pages describe as a paged-KV backend,
+ * "Inference-time context sparsity", sec. 1, "sparsity is usable for systems gains"):
+ *   q           bf16 [B][Hq][d]                          (raw 16-bit patterns)
+ *   K, V        bf16 [num_pages][P][Hkv][d]              (raw 16-bit patterns)
+ *   page_table  int32 [B][max_pages]; logical position p of request b lives in page
+ *               page_table[b][p / P], slot p % P
+ *   lens        int32 [B]  (N_b)
+ *   k           int32 [B]  (k_b; k_b >= N_b selects every row)
+ *   idx         int32 [B][Hq][k_max], ascending positions, -1 after the first min(k_b,N_b)
+ * Query head h reads KV head h / G with G = Hq / Hkv (contiguous GQA groups).
+ *
+ * Every entry point returns 0 on success and a negative number for an argument it cannot
+ * honour (it never reads outside the buffers it was given).
+ */
+#include <math.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* bf16 -> double is exact: a bf16 is the top half of an IEEE binary32. */
+static double bf16_to_double(uint16_t bits) {
+    uint32_t u = ((uint32_t)bits) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+typedef struct {
+    int B, Hq, Hkv, d, P, max_pages, k_max, num_pages;
+} oshape;
+
+static int check_shape(const oshape* s) {
+    if (s->B < 0 || s->Hq <= 0 || s->Hkv <= 0 || s->d <= 0 || s->P <= 0) return -1;
+    if (s->Hq % s->Hkv != 0) return -1;
+    if (s->max_pages < 0 || s->k_max < 0 || s->num_pages < 0) return -1;
+    return 0;
+}
+
+/* Pointer to row (b, kvh, logical position p) of a paged cache, or NULL if the page table
+ * points outside the cache. */
+static const uint16_t* cache_row(const oshape* s, const uint16_t* cache, const int32_t* page_table,
+                                 int b, int kvh, long p) {
+    long page_slot = p / s->P;
+    if (page_slot >= s->max_pages) return NULL;
+    int32_t page = page_table[(long)b * s->max_pages + page_slot];
+    if (page < 0 || page >= s->num_pages) return NULL;
+    long slot = p % s->P;
+    long row = ((long)page * s->P + slot) * s->Hkv + kvh;
+    return cache + row * s->d;
+}
+
+static int req_len(const oshape* s, const int32_t* lens, int b) {
+    int n = lens[b];
+    if (n < 0 || (long)n > (long)s->max_pages * s->P) return -1;
+    return n;
+}
+
+/* s[i] = q[b,h] . K[b, h/G, i] for i < N_b, in double. */
+static int scores_one(const oshape* s, const uint16_t* q, const uint16_t* K, const int32_t* page_table,
+                      int b, int h, int n, double* out) {
+    int G = s->Hq / s->Hkv;
+    int kvh = h / G;
+    const uint16_t* qh = q + ((long)b * s->Hq + h) * s->d;
+    for (long i = 0; i < n; ++i) {
+        const uint16_t* krow = cache_row(s, K, page_table, b, kvh, i);
+        if (!krow) return -2;
+        double acc = 0.0;
+        for (int j = 0; j < s->d; ++j) acc += bf16_to_double(qh[j]) * bf16_to_double(krow[j]);
+        out[i] = acc;
+    }
+    return 0;
+}
+
+int oracle_scores(int B, int Hq, int Hkv, int d, int P, int max_pages, int num_pages,
+                  const uint16_t* q, const uint16_t* K, const int32_t* page_table, const int32_t* lens,
+                  int b, int h, double* out) {
+    oshape s = {B, Hq, Hkv, d, P, max_pages, 0, num_pages};
+    if (check_shape(&s) || b < 0 || b >= B || h < 0 || h >= Hq) return -1;
+    int n = req_len(&s, lens, b);
+    if (n < 0) return -1;
+    return scores_one(&s, q, K, page_table, b, h, n, out);
+}
+
+/* Order used for selection: larger score first; equal scores -> lower position first.
+ * -0.0 and +0.0 compare equal (C's == on doubles). */
+typedef struct { double s; int32_t pos; } scored;
+
+static int by_score_then_pos(const void* a, const void* b) {
+    const scored* x = (const scored*)a;
+    const scored* y = (const scored*)b;
+    if (x->s > y->s) return -1;
+    if (x->s < y->s) return 1;
+    return (x->pos < y->pos) ? -1 : (x->pos > y->pos);
+}
+
+static int by_pos(const void* a, const void* b) {
+    int32_t x = *(const int32_t*)a, y = *(const int32_t*)b;
+    return (x < y) ? -1 : (x > y);
+}
+
+/* Exact top-k of one (b, h): writes min(k, n) ascending positions then -1 up to k_max. */
+static int topk_one(const oshape* s, const uint16_t* q, const uint16_t* K, const int32_t* page_table,
+                    int b, int h, int n, int kb, int32_t* idx_row) {
+    int take = kb < n ? kb : n;
+    if (take > s->k_max) return -3;
+    for (int i = 0; i < s->k_max; ++i) idx_row[i] = -1;
+    if (take <= 0) return 0;
+    double* sc = (double*)malloc(sizeof(double) * (size_t)n);
+    scored* all = (scored*)malloc(sizeof(scored) * (size_t)n);
+    if (!sc || !all) { free(sc); free(all); return -4; }
+    int rc = scores_one(s, q, K, page_table, b, h, n, sc);
+    if (rc == 0) {
+        for (int i = 0; i < n; ++i) { all[i].s = sc[i]; all[i].pos = i; }
+        qsort(all, (size_t)n, sizeof(scored), by_score_then_pos);
+        for (int i = 0; i < take; ++i) idx_row[i] = all[i].pos;
+        qsort(idx_row, (size_t)take, sizeof(int32_t), by_pos);
+    }
+    free(sc);
+    free(all);
+    return rc;
+}
+
+int oracle_topk(int B, int Hq, int Hkv, int d, int P, int max_pages, int num_pages, int k_max,
+                const uint16_t* q, const uint16_t* K, const int32_t* page_table, const int32_t* lens,
+                const int32_t* k, int32_t* idx) {
+    oshape s = {B, Hq, Hkv, d, P, max_pages, k_max, num_pages};
+    if (check_shape(&s)) return -1;
+    for (int b = 0; b < B; ++b) {
+        if (req_len(&s, lens, b) < 0) return -1;
+        if (k[b] < 1) return -1;
+    }
+    int rc_all = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(min : rc_all)
+    for (long bh = 0; bh < (long)B * Hq; ++bh) {
+        int b = (int)(bh / Hq), h = (int)(bh % Hq);
+        int rc = topk_one(&s, q, K, page_table, b, h, lens[b], k[b], idx + bh * (long)k_max);
+        if (rc < rc_all) rc_all = rc;
+    }
+    return rc_all;
+}
+
+/* Softmax attention of one (b, h) over the listed positions (order irrelevant):
+ * z_i = s_i / sqrt(d), w_i = exp(z_i - max z), out = sum w_i V_i / sum w_i.
+ * An empty list gives out = 0. */
+static int attend_one(const oshape* s, const uint16_t* q, const uint16_t* K, const uint16_t* V,
+                      const int32_t* page_table, int b, int h, int n, const int32_t* sel, int nsel,
+                      double* out) {
+    int G = s->Hq / s->Hkv;
+    int kvh = h / G;
+    const uint16_t* qh = q + ((long)b * s->Hq + h) * s->d;
+    for (int j = 0; j < s->d; ++j) out[j] = 0.0;
+    if (nsel == 0) return 0;
+    double* z = (double*)malloc(sizeof(double) * (size_t)nsel);
+    if (!z) return -4;
+    double scale = 1.0 / sqrt((double)s->d);
+    double zmax = -INFINITY;
+    for (int t = 0; t < nsel; ++t) {
+        int32_t p = sel[t];
+        if (p < 0 || p >= n) { free(z); return -2; }
+        const uint16_t* krow = cache_row(s, K, page_table, b, kvh, p);
+        if (!krow) { free(z); return -2; }
+        double acc = 0.0;
+        for (int j = 0; j < s->d; ++j) acc += bf16_to_double(qh[j]) * bf16_to_double(krow[j]);
+        z[t] = acc * scale;
+        if (z[t] > zmax) zmax = z[t];
+    }
+    double denom = 0.0;
+    for (int t = 0; t < nsel; ++t) {
+        double w = exp(z[t] - zmax);
+        const uint16_t* vrow = cache_row(s, V, page_table, b, kvh, sel[t]);
+        if (!vrow) { free(z); return -2; }
+        denom += w;
+        for (int j = 0; j < s->d; ++j) out[j] += w * bf16_to_double(vrow[j]);
+    }
+    for (int j = 0; j < s->d; ++j) out[j] /= denom;
+    free(z);
+    return 0;
+}
+
+/* Attention over the rows each (b, h) lists in idx (entries < 0 are padding and are skipped).
+ * out is double [B][Hq][d]. */
+int oracle_attend(int B, int Hq, int Hkv, int d, int P, int max_pages, int num_pages, int k_max,
+                  const uint16_t* q, const uint16_t* K, const uint16_t* V, const int32_t* page_table,
+                  const int32_t* lens, const int32_t* idx, double* out) {
+    oshape s = {B, Hq, Hkv, d, P, max_pages, k_max, num_pages};
+    if (check_shape(&s)) return -1;
+    for (int b = 0; b < B; ++b)
+        if (req_len(&s, lens, b) < 0) return -1;
+    int rc_all = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(min : rc_all)
+    for (long bh = 0; bh < (long)B * Hq; ++bh) {
+        int b = (int)(bh / Hq), h = (int)(bh % Hq);
+        const int32_t* row = idx + bh * (long)k_max;
+        int32_t* sel = (int32_t*)malloc(sizeof(int32_t) * (size_t)(k_max > 0 ? k_max : 1));
+        int nsel = 0;
+        int rc = sel ? 0 : -4;
+        if (sel) {
+            for (int t = 0; t < k_max; ++t)
+                if (row[t] >= 0) sel[nsel++] = row[t];
+            rc = attend_one(&s, q, K, V, page_table, b, h, lens[b], sel, nsel, out + bh * (long)d);
+        }
+        free(sel);
+        if (rc < rc_all) rc_all = rc;
+    }
+    return rc_all;
+}
+
+/* Dense decode: attention over every position 0..N_b-1.  out is double [B][Hq][d]. */
+int oracle_dense(int B, int Hq, int Hkv, int d, int P, int max_pages, int num_pages,
+                 const uint16_t* q, const uint16_t* K, const uint16_t* V, const int32_t* page_table,
+                 const int32_t* lens, double* out) {
+    oshape s = {B, Hq, Hkv, d, P, max_pages, 0, num_pages};
+    if (check_shape(&s)) return -1;
+    for (int b = 0; b < B; ++b)
+        if (req_len(&s, lens, b) < 0) return -1;
+    int rc_all = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(min : rc_all)
+    for (long bh = 0; bh < (long)B * Hq; ++bh) {
+        int b = (int)(bh / Hq), h = (int)(bh % Hq);
+        int n = lens[b];
+        int32_t* sel = (int32_t*)malloc(sizeof(int32_t) * (size_t)(n > 0 ? n : 1));
+        int rc = sel ? 0 : -4;
+        if (sel) {
+            for (int i = 0; i < n; ++i) sel[i] = i;
+            rc = attend_one(&s, q, K, V, page_table, b, h, n, sel, n, out + bh * (long)d);
+        }
+        free(sel);
+        if (rc < rc_all) rc_all = rc;
+    }
+    return rc_all;
+}
+
+/* Number of OpenMP threads the entry points above use (reported beside CPU timings). */
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

@@ -1,0 +1,67 @@
+"""The oracle pins must catch plausible mistakes.
+
+Each case below plants one mistake in a temporary copy of oracle/oracle.c (a dropped term, a wrong
+sign or index, a transposed layout, a reversed order), builds it with gcc, routes the oracle module
+through that copy, and checks that at least one pin of tests/test_oracle.py fails.  The real oracle
+is never modified.  CPU only.
+"""
+from __future__ import annotations
+
+import os
+
+import pytest
+
+import oracle
+from tests import test_oracle as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
+
+# (name, exact text in oracle.c, replacement)
+MUTANTS = [
+    ("drop_softmax_scale", "double scale = 1.0 / sqrt((double)s->d);", "double scale = 1.0;"),
+    ("gqa_modulo_mapping", "int kvh = h / G;", "int kvh = h % s->Hkv;"),
+    ("ties_to_higher_position", "return (x->pos < y->pos) ? -1 : (x->pos > y->pos);",
+     "return (x->pos > y->pos) ? -1 : (x->pos < y->pos);"),
+    ("select_smallest", "if (x->s > y->s) return -1;\n    if (x->s < y->s) return 1;",
+     "if (x->s < y->s) return -1;\n    if (x->s > y->s) return 1;"),
+    ("hnd_instead_of_nhd", "long row = ((long)page * s->P + slot) * s->Hkv + kvh;",
+     "long row = ((long)page * s->Hkv + kvh) * s->P + slot;"),
+    ("slot_from_wrong_axis", "long slot = p % s->P;", "long slot = (p / s->P) % s->P;"),
+    ("drop_first_dim", "for (int j = 0; j < s->d; ++j) acc += bf16_to_double(qh[j]) * bf16_to_double(krow[j]);\n        out[i]",
+     "for (int j = 1; j < s->d; ++j) acc += bf16_to_double(qh[j]) * bf16_to_double(krow[j]);\n        out[i]"),
+    ("no_normalisation", "for (int j = 0; j < s->d; ++j) out[j] /= denom;", ""),
+    ("sign_flip_in_exponent", "double w = exp(z[t] - zmax);", "double w = exp(zmax - z[t]);"),
+    ("one_row_short", "for (int i = 0; i < take; ++i) idx_row[i] = all[i].pos;",
+     "for (int i = 0; i + 1 < take; ++i) idx_row[i] = all[i].pos;"),
+    ("unsorted_output", "qsort(idx_row, (size_t)take, sizeof(int32_t), by_pos);", ""),
+]
+
+PINS = [
+    pins.test_golden_topk_ties,
+    pins.test_topk_brute_force_tiny,
+    pins.test_topk_brute_force_random_real_scores,
+    pins.test_scores_closed_form_paging_and_gqa,
+    pins.test_dense_equals_library_sdpa,
+    pins.test_any_k_equals_masked_library_sdpa,
+    pins.test_k1_returns_argmax_row,
+    pins.test_two_rows_logistic_closed_form,
+    pins.test_golden_uniform_average,
+]
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_reject_mutant(tmp_path, name, old, new):
+    src = open(SRC).read()
+    assert src.count(old) >= 1, f"mutation site for {name} not found"
+    mutated = src.replace(old, new)
+    path = tmp_path / "oracle_mut.c"
+    path.write_text(mutated)
+    lib = oracle.compile_source(str(path), str(tmp_path / "liboracle_mut.so"))
+    failed = []
+    with oracle.use_library(lib):
+        for pin in PINS:
+            try:
+                pin()
+            except (AssertionError, ValueError):
+                failed.append(pin.__name__)
+    assert failed, f"no pin caught mutant {name}"
