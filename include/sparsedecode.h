@@ -1,0 +1,151 @@
+/*
+ * sparsedecode.h -- C ABI of libsparsedecode: exact top-k sparse decode attention over a paged,
+ * grouped-query (GQA), bf16 KV cache, on NVIDIA B200 (sm_100a).
+ *
+ * The method (sources are the pages' titles and sections):
+ *   - "Technische Zusammenfassung: Kontextsparsitaet bei der Inferenzzeit - Illusion oder
+ *     Chance?", sec. 2, "Sparsitaetsmechanismen: Oracle Top-K": an exact top-k indexer picks, per
+ *     decode query and query head, the k keys with the highest score q.K.
+ *   - "Inference-time context sparsity: illusion or opportunity?", Fig. 1(a): dense decode reads
+ *     O(N d) bytes per step, sparse decode routes through an indexer that keeps k rows and reads
+ *     O(k d) bytes; sec. 1 ("sparsity is usable for systems gains"): the kernels handle sparsity
+ *     that is irregular per token, per query and per head, under GQA, over a paged KV cache.
+ *   - "Sparse Attention inference survey" (xllm), sec. 1.1: scaled dot-product attention,
+ *     softmax(q K^T / sqrt(d)) V; here evaluated over the selected rows only, so the softmax is
+ *     renormalised over the selected set.
+ *
+ * Conventions shared by every entry point
+ *   Shapes      B requests, Hq query heads, Hkv KV heads, G = Hq / Hkv (1 <= G <= 16), head
+ *               dimension d = 128, page size P = 16.  Query head h reads KV head h / G.
+ *   q           bf16 [B][Hq][d], row-major, device memory, 16-byte aligned.
+ *   K, V        bf16 [num_pages][P][Hkv][d] ("NHD" pages), device memory, 16-byte aligned.
+ *               Logical position p of request b is row [page_table[b][p / P]][p % P].
+ *   page_table  int32 [B][max_pages_per_req], device memory.  Entries at positions >= lens[b]
+ *               are never read.
+ *   lens        int32 [B], device memory: context length N_b, 0 <= N_b <= max_pages_per_req * P.
+ *   idx         int32 [B][Hq][k_max], device memory: per (b, h) the selected positions in strictly
+ *               ascending order, followed by -1 padding.  Any negative entry counts as padding.
+ *   out         fp32 [B][Hq][d], device memory, 16-byte aligned.
+ *   workspace   device scratch owned by the caller, at least sd_workspace_size() bytes,
+ *               256-byte aligned.  Its contents need no initialisation and are not preserved.
+ *   dev_status  int32, device memory, owned by the caller and zeroed by the caller.  Kernels
+ *               never trap: a violated device-side precondition (bad length, bad k, an index or
+ *               page entry out of range) makes the first failing kernel store its sd_status code
+ *               there (first error wins; later calls keep it) and skip the offending access.
+ *               Read it after synchronising the stream.  Outputs of a call that set it are
+ *               unspecified.
+ *   stream      a cudaStream_t passed as void*; NULL means the legacy default stream.  Every
+ *               call is asynchronous on that stream, uses the current CUDA device, allocates
+ *               nothing and keeps no state between calls.
+ *   Return      host-side validation happens before any launch; a non-SD_OK return means nothing
+ *               was launched (SD_ERR_CUDA: a launch failed; the CUDA error is not cleared).
+ */
+#ifndef SPARSEDECODE_H
+#define SPARSEDECODE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SD_API __attribute__((visibility("default")))
+#else
+#define SD_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct sd_shape {
+    int32_t batch;              /* B, >= 1 */
+    int32_t num_q_heads;        /* Hq, >= 1, multiple of num_kv_heads */
+    int32_t num_kv_heads;       /* Hkv, >= 1, Hq / Hkv <= 16 */
+    int32_t head_dim;           /* d; only 128 is supported */
+    int32_t page_size;          /* P; only 16 is supported */
+    int32_t max_pages_per_req;  /* row length of page_table, >= 1 */
+    int32_t k_max;              /* row length of idx, >= 1 */
+    int32_t num_pages;          /* pages in each of K and V, >= 1 */
+} sd_shape;
+
+typedef int32_t sd_status;
+
+enum {
+    SD_OK = 0,
+    SD_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, inconsistent shape, bad length or k */
+    SD_ERR_UNSUPPORTED = 2,   /* head_dim != 128, page_size != 16, G > 16, sizes beyond limits */
+    SD_ERR_CUDA = 3,          /* a CUDA runtime call or kernel launch failed */
+    SD_ERR_INDEX_OOB = 4,     /* device: idx entry >= N_b, or page entry outside [0, num_pages) */
+    SD_ERR_TIMEOUT = 5,       /* device: a bounded wait inside a kernel gave up */
+    SD_ERR_WORKSPACE = 6,     /* workspace_bytes smaller than sd_workspace_size() */
+    SD_ERR_ORDER = 7          /* device: an idx row is not strictly ascending */
+};
+
+enum { SD_OP_TOPK = 1, SD_OP_SPARSE = 2, SD_OP_DENSE = 3 };
+
+/* Bytes of workspace that operation `op` needs for `shape` (independent of the data and of the
+ * device).  Returns SD_ERR_INVALID_ARG / SD_ERR_UNSUPPORTED for a shape the library rejects. */
+SD_API sd_status sd_workspace_size(const sd_shape* shape, int32_t op, size_t* bytes);
+
+/* Exact top-k indexer ("Oracle Top-K", gist.science summary sec. 2; the indexer of Fig. 1(a) of
+ * "Inference-time context sparsity").
+ *   For every request b and query head h: s_i = q[b,h] . K[b, h/G, i] for 0 <= i < N_b (fp32
+ *   accumulation of exact bf16 products); keep the min(k[b], N_b) positions with the largest s,
+ *   ties at the k-th score going to the lower position (-0.0 equals +0.0; NaN inputs are
+ *   invalid); write them to idx[b][h] in ascending order, then -1 up to k_max.
+ *   k       int32 [B], device memory, 1 <= k[b]; min(k[b], N_b) must not exceed k_max
+ *           (else SD_ERR_INVALID_ARG in dev_status and that row is left all -1).
+ *   Requests with k[b] >= N_b are returned as 0..N_b-1 without reading K. */
+SD_API sd_status sd_topk_index(const sd_shape* shape, const void* q, const void* K, const int32_t* page_table,
+                        const int32_t* lens, const int32_t* k, int32_t* idx, void* workspace,
+                        size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/* The two halves of sd_topk_index, for callers that schedule or time them separately.
+ *   sd_topk_scores  writes s[b][h][i] (fp32) for every request that needs a selection
+ *                   (1 <= k[b] < N_b) into the workspace; other rows are not written.
+ *   sd_topk_select  reads those scores from the same workspace and writes idx exactly as
+ *                   sd_topk_index does; it must follow sd_topk_scores on the same inputs and
+ *                   workspace (stream order), with lens and k unchanged in between. */
+SD_API sd_status sd_topk_scores(const sd_shape* shape, const void* q, const void* K, const int32_t* page_table,
+                         const int32_t* lens, const int32_t* k, void* workspace, size_t workspace_bytes,
+                         int32_t* dev_status, void* stream);
+SD_API sd_status sd_topk_select(const sd_shape* shape, const int32_t* lens, const int32_t* k, int32_t* idx,
+                         void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/* Sparse decode attention over the selected rows ("Sparse" mode of Fig. 1(a) of "Inference-time
+ * context sparsity"; SDPA of the xllm survey sec. 1.1 restricted to the selected set).
+ *   out[b,h] = sum_{i in S} w_i V[b, h/G, i],  w = softmax over S of (q[b,h] . K[b,h/G,i]) / sqrt(d),
+ *   S = the non-negative entries of idx[b][h].  An empty S gives out = 0.
+ *   Each GQA group reads the union of its heads' selected rows once.
+ *   Device checks: entries must be < N_b (SD_ERR_INDEX_OOB) and strictly ascending
+ *   (SD_ERR_ORDER). */
+SD_API sd_status sd_sparse_decode(const sd_shape* shape, const void* q, const void* K, const void* V,
+                           const int32_t* page_table, const int32_t* lens, const int32_t* idx, float* out,
+                           void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/* Dense decode attention over all N_b rows ("Dense" mode of Fig. 1(a)); the comparator of the
+ * sparse kernel at the same shape.  shape->k_max is ignored. */
+SD_API sd_status sd_dense_decode(const sd_shape* shape, const void* q, const void* K, const void* V,
+                          const int32_t* page_table, const int32_t* lens, float* out, void* workspace,
+                          size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/* Append one decode step's K/V row per request (the growing cache of an agentic decode loop).
+ *   For each b: p = lens[b]; the rows k_new[b][kvh][:] and v_new[b][kvh][:] (bf16 [B][Hkv][d],
+ *   device memory) are written to K and V at position p through page_table; then lens[b] = p + 1
+ *   and, if k_sel is not NULL, k_sel[b] = max(1, round_half_up((p + 1) / ratio)).
+ *   p must satisfy p < max_pages_per_req * P and its page entry must be in range, else the row is
+ *   not written, lens[b] is unchanged and dev_status records the error.  ratio >= 1. */
+SD_API sd_status sd_append_kv(const sd_shape* shape, void* K, void* V, const int32_t* page_table, int32_t* lens,
+                       const void* k_new, const void* v_new, int32_t* k_sel, int32_t ratio,
+                       int32_t* dev_status, void* stream);
+
+/* Static English text for a status code ("unknown status" for other values). */
+SD_API const char* sd_status_string(sd_status status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+SD_API int32_t sd_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPARSEDECODE_H */

@@ -1,0 +1,293 @@
+// api.cu -- the C ABI of libsparsedecode (declared in include/sparsedecode.h): host-side argument
+// validation, workspace layout, launch configuration and status codes.  No allocation, no state
+// beyond a per-device cache of the SM count and decode occupancy.
+#include <math.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace sd;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr size_t kSmemBudget = 227 * 1024;   // opt-in shared memory per CTA on sm_100
+constexpr int kSelectCapMax = 24 * 1024;      // select: candidate entries kept in shared memory
+
+struct DeviceInfo {
+    bool ready = false;
+    int sms = 0;
+    int decode_ctas_per_sm = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+
+sd_status device_info(DeviceInfo* out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SD_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return SD_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceInfo& d = g_dev[dev];
+    if (!d.ready) {
+        int sms = 0, ctas = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return SD_ERR_CUDA;
+        if (decode_occupancy(&ctas) != cudaSuccess || ctas < 1) return SD_ERR_CUDA;
+        d.sms = sms;
+        d.decode_ctas_per_sm = ctas;
+        d.ready = true;
+    }
+    *out = d;
+    return SD_OK;
+}
+
+struct Dims {
+    int B, Hq, Hkv, G, max_pages, k_max, num_pages;
+    long n_cap;   // max_pages * page size
+    int n_gran;   // 128-position granules of n_cap
+    int jmax;     // decode segment slots per (b, h)
+};
+
+sd_status check_shape(const sd_shape* s, Dims* d) {
+    if (s == nullptr) return SD_ERR_INVALID_ARG;
+    if (s->batch < 1 || s->num_q_heads < 1 || s->num_kv_heads < 1 || s->max_pages_per_req < 1 || s->k_max < 1 ||
+        s->num_pages < 1)
+        return SD_ERR_INVALID_ARG;
+    if (s->num_q_heads % s->num_kv_heads != 0) return SD_ERR_INVALID_ARG;
+    if (s->head_dim != kHeadDim || s->page_size != kPageSize) return SD_ERR_UNSUPPORTED;
+    const int G = s->num_q_heads / s->num_kv_heads;
+    if (G > kMaxGroup || s->num_kv_heads > 16 || s->batch > kMaxBatch) return SD_ERR_UNSUPPORTED;
+    const long n_cap = (long)s->max_pages_per_req * kPageSize;
+    if (n_cap > (1L << 30)) return SD_ERR_UNSUPPORTED;
+    if ((long)s->num_pages * kPageSize * s->num_kv_heads >= (1L << 32)) return SD_ERR_UNSUPPORTED;   // row index is 32-bit
+    d->B = s->batch;
+    d->Hq = s->num_q_heads;
+    d->Hkv = s->num_kv_heads;
+    d->G = G;
+    d->max_pages = s->max_pages_per_req;
+    d->k_max = s->k_max;
+    d->num_pages = s->num_pages;
+    d->n_cap = n_cap;
+    d->n_gran = (int)((n_cap + 127) / 128);
+    d->jmax = d->n_gran + 1;
+    return SD_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+size_t topk_workspace(const Dims& d) { return align256((size_t)d.B * d.Hq * d.n_cap * sizeof(float)); }
+
+// decode workspace: acc [B][Hq][jmax][128] fp32, then ml [B][Hq][jmax] float2
+size_t decode_acc_bytes(const Dims& d) { return align256((size_t)d.B * d.Hq * d.jmax * kHeadDim * sizeof(float)); }
+size_t decode_workspace(const Dims& d) { return decode_acc_bytes(d) + align256((size_t)d.B * d.Hq * d.jmax * sizeof(float2)); }
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+sd_status launch_status(cudaError_t e) { return e == cudaSuccess ? SD_OK : SD_ERR_CUDA; }
+
+sd_status decode_common(const sd_shape* shape, const void* q, const void* K, const void* V, const int32_t* page_table,
+                        const int32_t* lens, const int32_t* idx, float* out, void* workspace, size_t workspace_bytes,
+                        int32_t* dev_status, void* stream, bool dense) {
+    Dims d;
+    sd_status st = check_shape(shape, &d);
+    if (st != SD_OK) return st;
+    if (!q || !K || !V || !page_table || !lens || !out || !workspace || !dev_status || (!dense && !idx))
+        return SD_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(out, 16) || !aligned(workspace, 256) ||
+        !aligned(page_table, 4) || !aligned(lens, 4) || (!dense && !aligned(idx, 4)) || !aligned(dev_status, 4))
+        return SD_ERR_INVALID_ARG;
+    if (workspace_bytes < decode_workspace(d)) return SD_ERR_WORKSPACE;
+    DeviceInfo di;
+    st = device_info(&di);
+    if (st != SD_OK) return st;
+    DecodeArgs a;
+    a.q = static_cast<const __nv_bfloat16*>(q);
+    a.K = static_cast<const __nv_bfloat16*>(K);
+    a.V = static_cast<const __nv_bfloat16*>(V);
+    a.page_table = page_table;
+    a.lens = lens;
+    a.idx = dense ? nullptr : idx;
+    a.out = out;
+    a.acc = static_cast<float*>(workspace);
+    a.ml = reinterpret_cast<float2*>(static_cast<uint8_t*>(workspace) + decode_acc_bytes(d));
+    a.status = dev_status;
+    a.B = d.B;
+    a.Hq = d.Hq;
+    a.Hkv = d.Hkv;
+    a.G = d.G;
+    a.max_pages = d.max_pages;
+    a.num_pages = d.num_pages;
+    a.k_max = dense ? 0 : d.k_max;
+    a.n_cap = d.n_cap;
+    a.jmax = d.jmax;
+    const int ctas = di.sms * di.decode_ctas_per_sm;
+    a.total_warps = ctas * kDecodeWarpsPerCta;
+    a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)kHeadDim));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    st = launch_status(launch_decode(a, dense, ctas, s));
+    if (st != SD_OK) return st;
+    return launch_status(launch_merge(a, s));
+}
+
+}  // namespace
+
+extern "C" {
+
+sd_status sd_workspace_size(const sd_shape* shape, int32_t op, size_t* bytes) {
+    if (bytes == nullptr) return SD_ERR_INVALID_ARG;
+    Dims d;
+    sd_status st = check_shape(shape, &d);
+    if (st != SD_OK) return st;
+    switch (op) {
+        case SD_OP_TOPK: *bytes = topk_workspace(d); return SD_OK;
+        case SD_OP_SPARSE:
+        case SD_OP_DENSE: *bytes = decode_workspace(d); return SD_OK;
+        default: return SD_ERR_INVALID_ARG;
+    }
+}
+
+namespace {
+
+sd_status topk_args(const sd_shape* shape, const void* q, const void* K, const int32_t* page_table,
+                    const int32_t* lens, const int32_t* k, int32_t* idx, void* workspace, size_t workspace_bytes,
+                    int32_t* dev_status, bool need_scores_inputs, bool need_idx, TopkArgs* a, DeviceInfo* di) {
+    Dims d;
+    sd_status st = check_shape(shape, &d);
+    if (st != SD_OK) return st;
+    if (!lens || !k || !workspace || !dev_status) return SD_ERR_INVALID_ARG;
+    if (need_scores_inputs && (!q || !K || !page_table)) return SD_ERR_INVALID_ARG;
+    if (need_idx && !idx) return SD_ERR_INVALID_ARG;
+    if ((need_scores_inputs && (!aligned(q, 16) || !aligned(K, 16) || !aligned(page_table, 4))) ||
+        (need_idx && !aligned(idx, 4)) || !aligned(workspace, 256) || !aligned(lens, 4) || !aligned(k, 4) ||
+        !aligned(dev_status, 4))
+        return SD_ERR_INVALID_ARG;
+    if (workspace_bytes < topk_workspace(d)) return SD_ERR_WORKSPACE;
+    st = device_info(di);
+    if (st != SD_OK) return st;
+    a->q = static_cast<const __nv_bfloat16*>(q);
+    a->K = static_cast<const __nv_bfloat16*>(K);
+    a->page_table = page_table;
+    a->lens = lens;
+    a->k = k;
+    a->idx = idx;
+    a->scores = static_cast<float*>(workspace);
+    a->status = dev_status;
+    a->B = d.B;
+    a->Hq = d.Hq;
+    a->Hkv = d.Hkv;
+    a->G = d.G;
+    a->max_pages = d.max_pages;
+    a->num_pages = d.num_pages;
+    a->k_max = d.k_max;
+    a->n_cap = d.n_cap;
+    // score pass: pipeline stages of >= 32 KB, as deep as the shared memory allows (<= 6)
+    const size_t page_bytes = (size_t)kPageSize * d.Hkv * kRowBytes;
+    a->spp = (int)(page_bytes >= 32768 ? 1 : 32768 / page_bytes);
+    const size_t fixed = sizeof(int) * (d.B + 1 + 40) + 1024;
+    const size_t stage_bytes = page_bytes * a->spp;
+    a->stages = (int)((kSmemBudget - fixed) / (stage_bytes + 2 * sizeof(uint64_t)));
+    if (a->stages > 6) a->stages = 6;
+    if (a->stages < 2) return SD_ERR_UNSUPPORTED;
+    // select: candidate capacity from k_max, bounded by shared memory
+    long cap = (long)d.k_max + d.k_max / 2 + 4096;
+    if (cap > kSelectCapMax) cap = kSelectCapMax;
+    a->cap = (int)cap;
+    return SD_OK;
+}
+
+}  // namespace
+
+sd_status sd_topk_scores(const sd_shape* shape, const void* q, const void* K, const int32_t* page_table,
+                         const int32_t* lens, const int32_t* k, void* workspace, size_t workspace_bytes,
+                         int32_t* dev_status, void* stream) {
+    TopkArgs a;
+    DeviceInfo di;
+    sd_status st = topk_args(shape, q, K, page_table, lens, k, nullptr, workspace, workspace_bytes, dev_status, true,
+                             false, &a, &di);
+    if (st != SD_OK) return st;
+    return launch_status(launch_score_pass(a, di.sms, static_cast<cudaStream_t>(stream)));
+}
+
+sd_status sd_topk_select(const sd_shape* shape, const int32_t* lens, const int32_t* k, int32_t* idx, void* workspace,
+                         size_t workspace_bytes, int32_t* dev_status, void* stream) {
+    TopkArgs a;
+    DeviceInfo di;
+    sd_status st = topk_args(shape, nullptr, nullptr, nullptr, lens, k, idx, workspace, workspace_bytes, dev_status,
+                             false, true, &a, &di);
+    if (st != SD_OK) return st;
+    return launch_status(launch_select(a, static_cast<cudaStream_t>(stream)));
+}
+
+sd_status sd_topk_index(const sd_shape* shape, const void* q, const void* K, const int32_t* page_table,
+                        const int32_t* lens, const int32_t* k, int32_t* idx, void* workspace, size_t workspace_bytes,
+                        int32_t* dev_status, void* stream) {
+    TopkArgs a;
+    DeviceInfo di;
+    sd_status st = topk_args(shape, q, K, page_table, lens, k, idx, workspace, workspace_bytes, dev_status, true, true,
+                             &a, &di);
+    if (st != SD_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    st = launch_status(launch_score_pass(a, di.sms, s));
+    if (st != SD_OK) return st;
+    return launch_status(launch_select(a, s));
+}
+
+sd_status sd_sparse_decode(const sd_shape* shape, const void* q, const void* K, const void* V,
+                           const int32_t* page_table, const int32_t* lens, const int32_t* idx, float* out,
+                           void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream) {
+    return decode_common(shape, q, K, V, page_table, lens, idx, out, workspace, workspace_bytes, dev_status, stream,
+                         false);
+}
+
+sd_status sd_dense_decode(const sd_shape* shape, const void* q, const void* K, const void* V,
+                          const int32_t* page_table, const int32_t* lens, float* out, void* workspace,
+                          size_t workspace_bytes, int32_t* dev_status, void* stream) {
+    return decode_common(shape, q, K, V, page_table, lens, nullptr, out, workspace, workspace_bytes, dev_status,
+                         stream, true);
+}
+
+sd_status sd_append_kv(const sd_shape* shape, void* K, void* V, const int32_t* page_table, int32_t* lens,
+                       const void* k_new, const void* v_new, int32_t* k_sel, int32_t ratio, int32_t* dev_status,
+                       void* stream) {
+    Dims d;
+    sd_status st = check_shape(shape, &d);
+    if (st != SD_OK) return st;
+    if (!K || !V || !page_table || !lens || !k_new || !v_new || !dev_status || ratio < 1) return SD_ERR_INVALID_ARG;
+    if (!aligned(K, 16) || !aligned(V, 16) || !aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(page_table, 4) ||
+        !aligned(lens, 4) || (k_sel && !aligned(k_sel, 4)) || !aligned(dev_status, 4))
+        return SD_ERR_INVALID_ARG;
+    AppendArgs a;
+    a.K = static_cast<__nv_bfloat16*>(K);
+    a.V = static_cast<__nv_bfloat16*>(V);
+    a.page_table = page_table;
+    a.lens = lens;
+    a.k_new = static_cast<const __nv_bfloat16*>(k_new);
+    a.v_new = static_cast<const __nv_bfloat16*>(v_new);
+    a.k_sel = k_sel;
+    a.status = dev_status;
+    a.B = d.B;
+    a.Hkv = d.Hkv;
+    a.max_pages = d.max_pages;
+    a.num_pages = d.num_pages;
+    a.ratio = ratio;
+    return launch_status(launch_append(a, static_cast<cudaStream_t>(stream)));
+}
+
+const char* sd_status_string(sd_status status) {
+    switch (status) {
+        case SD_OK: return "ok";
+        case SD_ERR_INVALID_ARG: return "invalid argument";
+        case SD_ERR_UNSUPPORTED: return "unsupported shape or size";
+        case SD_ERR_CUDA: return "CUDA error";
+        case SD_ERR_INDEX_OOB: return "index or page entry out of range";
+        case SD_ERR_TIMEOUT: return "bounded wait in a kernel gave up";
+        case SD_ERR_WORKSPACE: return "workspace too small";
+        case SD_ERR_ORDER: return "index row not strictly ascending";
+        default: return "unknown status";
+    }
+}
+
+int32_t sd_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,69 @@
+// kernels.h -- internal interface between the C-ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace sd {
+
+struct TopkArgs {
+    const __nv_bfloat16* q;
+    const __nv_bfloat16* K;
+    const int32_t* page_table;
+    const int32_t* lens;
+    const int32_t* k;
+    int32_t* idx;
+    float* scores;      // workspace: fp32 [B][Hq][n_cap]
+    int32_t* status;
+    int B, Hq, Hkv, G, max_pages, num_pages, k_max;
+    long n_cap;         // max_pages * page size: row stride of the score buffer
+    int spp;            // pages per pipeline stage of the score pass
+    int stages;         // pipeline depth of the score pass
+    int cap;            // select: candidate entries that fit in shared memory
+};
+
+size_t score_pass_smem(const TopkArgs& a);
+size_t select_smem(const TopkArgs& a);
+cudaError_t launch_score_pass(const TopkArgs& a, int grid, cudaStream_t stream);
+cudaError_t launch_select(const TopkArgs& a, cudaStream_t stream);
+
+struct DecodeArgs {
+    const __nv_bfloat16* q;
+    const __nv_bfloat16* K;
+    const __nv_bfloat16* V;
+    const int32_t* page_table;
+    const int32_t* lens;
+    const int32_t* idx;   // null for dense decode
+    float* out;
+    float2* ml;           // workspace: per (b, h, segment) running max (log2 units) and sum
+    float* acc;           // workspace: per (b, h, segment) un-normalised output [128]
+    int32_t* status;
+    int B, Hq, Hkv, G, max_pages, num_pages, k_max;
+    long n_cap;
+    int jmax;             // segment slots per (b, h)
+    int total_warps;      // persistent decode warps in the grid
+    float scale_log2;     // log2(e) / sqrt(d)
+};
+
+constexpr int kDecodeWarpsPerCta = 4;
+size_t decode_smem();
+cudaError_t decode_occupancy(int* ctas_per_sm);
+cudaError_t launch_decode(const DecodeArgs& a, bool dense, int ctas, cudaStream_t stream);
+cudaError_t launch_merge(const DecodeArgs& a, cudaStream_t stream);
+
+struct AppendArgs {
+    __nv_bfloat16* K;
+    __nv_bfloat16* V;
+    const int32_t* page_table;
+    int32_t* lens;
+    const __nv_bfloat16* k_new;
+    const __nv_bfloat16* v_new;
+    int32_t* k_sel;
+    int32_t* status;
+    int B, Hkv, max_pages, num_pages, ratio;
+};
+cudaError_t launch_append(const AppendArgs& a, cudaStream_t stream);
+
+}  // namespace sd

@@ -1,0 +1,128 @@
+"""The C-ABI library loads, exports every entry point its header declares, and validates arguments on
+the host before any launch.  CPU only: no call here reaches a kernel."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from sparse_attention_decode_sd_b200 import binding as sdb
+from sparse_attention_decode_sd_b200 import build as sdbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sparsedecode.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    sdbuild.build()
+    return sdb.load()
+
+
+def _declared():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"SD_API\s+[\w\s\*]+?\b(sd_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_names():
+    assert _declared() == sorted(sdb.EXPORTED)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", sdb.library_path()], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r"\sT\s(sd_\w+)$", out, flags=re.M))
+    for name in _declared():
+        assert name in exported, name
+        assert hasattr(lib, name)
+
+
+def test_header_compiles_as_c():
+    src = '#include "sparsedecode.h"\nint main(void){ sd_shape s; (void)s; return SD_OK; }\n'
+    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-fsyntax-only", "-I", os.path.dirname(HEADER), "-x",
+                        "c", "-"], input=src, text=True, capture_output=True)
+    assert r.returncode == 0, r.stderr
+
+
+def test_status_strings_and_version(lib):
+    assert sdb.status_string(sdb.SD_OK) == "ok"
+    for code in range(1, 8):
+        assert sdb.status_string(code) not in ("ok", "unknown status")
+    assert sdb.status_string(99) == "unknown status"
+    assert sdb.version() >= 100
+
+
+def _shape(**kw):
+    base = dict(B=4, Hq=64, Hkv=8, max_pages=8192, k_max=2621, num_pages=32768)
+    base.update(kw)
+    return sdb.make_shape(base["B"], base["Hq"], base["Hkv"], base["max_pages"], base["k_max"], base["num_pages"],
+                          base.get("head_dim", 128), base.get("page_size", 16))
+
+
+def test_workspace_sizes(lib):
+    s = _shape()
+    topk = sdb.sd_workspace_size(s, sdb.SD_OP_TOPK)
+    assert topk == 4 * 64 * 8192 * 16 * 4                  # fp32 scores [B][Hq][n_cap]
+    sparse = sdb.sd_workspace_size(s, sdb.SD_OP_SPARSE)
+    assert sparse == sdb.sd_workspace_size(s, sdb.SD_OP_DENSE)
+    slots = 4 * 64 * (8192 * 16 // 128 + 1)
+    assert sparse >= slots * (128 * 4 + 8)
+    assert sparse % 256 == 0 and topk % 256 == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(B=0), sdb.SD_ERR_INVALID_ARG),
+    (dict(Hq=60, Hkv=8), sdb.SD_ERR_INVALID_ARG),
+    (dict(k_max=0), sdb.SD_ERR_INVALID_ARG),
+    (dict(num_pages=0), sdb.SD_ERR_INVALID_ARG),
+    (dict(head_dim=64), sdb.SD_ERR_UNSUPPORTED),
+    (dict(page_size=32), sdb.SD_ERR_UNSUPPORTED),
+    (dict(Hq=136, Hkv=4), sdb.SD_ERR_UNSUPPORTED),   # G = 34 > 16
+    (dict(Hkv=32, Hq=64), sdb.SD_ERR_UNSUPPORTED),   # more than 16 KV heads
+])
+def test_shape_validation(lib, kw, code):
+    n = ctypes.c_size_t(0)
+    st = lib.sd_workspace_size(ctypes.byref(_shape(**kw)), sdb.SD_OP_SPARSE, ctypes.byref(n))
+    assert st == code
+
+
+def test_bad_op_and_null_shape(lib):
+    n = ctypes.c_size_t(0)
+    assert lib.sd_workspace_size(None, sdb.SD_OP_TOPK, ctypes.byref(n)) == sdb.SD_ERR_INVALID_ARG
+    assert lib.sd_workspace_size(ctypes.byref(_shape()), 9, ctypes.byref(n)) == sdb.SD_ERR_INVALID_ARG
+    assert lib.sd_workspace_size(ctypes.byref(_shape()), sdb.SD_OP_TOPK, None) == sdb.SD_ERR_INVALID_ARG
+
+
+def test_null_and_misaligned_pointers_rejected_before_launch(lib):
+    s = ctypes.byref(_shape())
+    fake = ctypes.c_void_p(1 << 20)       # never dereferenced: validation fails first
+    odd = ctypes.c_void_p((1 << 20) + 2)
+    N = None
+    ws = ctypes.c_size_t(1 << 40)
+    assert lib.sd_topk_index(s, N, fake, fake, fake, fake, fake, fake, ws, fake, N) == sdb.SD_ERR_INVALID_ARG
+    assert lib.sd_topk_index(s, odd, fake, fake, fake, fake, fake, fake, ws, fake, N) == sdb.SD_ERR_INVALID_ARG
+    assert lib.sd_sparse_decode(s, fake, fake, fake, fake, fake, N, fake, fake, ws, fake, N) == sdb.SD_ERR_INVALID_ARG
+    assert lib.sd_sparse_decode(s, fake, fake, odd, fake, fake, fake, fake, fake, ws, fake, N) == sdb.SD_ERR_INVALID_ARG
+    assert lib.sd_dense_decode(s, fake, fake, fake, fake, fake, fake, N, ws, fake, N) == sdb.SD_ERR_INVALID_ARG
+    assert lib.sd_append_kv(s, fake, fake, fake, fake, fake, fake, N, 0, fake, N) == sdb.SD_ERR_INVALID_ARG
+    assert lib.sd_append_kv(s, fake, fake, fake, fake, N, fake, N, 50, fake, N) == sdb.SD_ERR_INVALID_ARG
+
+
+def test_small_workspace_rejected_before_launch(lib):
+    s = ctypes.byref(_shape())
+    fake = ctypes.c_void_p(1 << 20)
+    small = ctypes.c_size_t(1024)
+    assert lib.sd_topk_index(s, fake, fake, fake, fake, fake, fake, fake, small, fake, None) == sdb.SD_ERR_WORKSPACE
+    assert lib.sd_sparse_decode(s, fake, fake, fake, fake, fake, fake, fake, fake, small, fake, None) == \
+        sdb.SD_ERR_WORKSPACE
+    assert lib.sd_dense_decode(s, fake, fake, fake, fake, fake, fake, fake, small, fake, None) == sdb.SD_ERR_WORKSPACE
+
+
+def test_library_does_not_link_the_oracle():
+    out = subprocess.run(["nm", "-D", sdb.library_path()], capture_output=True, text=True, check=True).stdout
+    assert "oracle_" not in out
+    ldd = subprocess.run(["ldd", sdb.library_path()], capture_output=True, text=True).stdout
+    assert "oracle" not in ldd

@@ -1,0 +1,246 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 CPU oracle on the same seeded inputs.
+
+Small cases are compared element by element on every (b, h); the full-size workloads (the five
+named configurations) run in the launch configuration the benchmark times and are compared on
+sampled (request, KV head) groups.  Rules and tolerances: tests/gpu_helpers.py.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sparse_attention_decode_sd_b200 import binding as sdb
+from sparse_attention_decode_sd_b200 import workloads as wl
+from tests import gpu_helpers as gh
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def _run_small(w_cpu, check_dense=True):
+    w = w_cpu.to(DEV)
+    r = gh.Runner(w)
+    return gh.full_parity(w_cpu, r, check_dense=check_dense)
+
+
+def test_tiny_planted_keys():
+    w_cpu = wl.named("tiny")
+    idx, _ = _run_small(w_cpu)
+    for (b, h), pos in w_cpu.meta["planted"].items():
+        assert set(pos.tolist()) <= set(idx[b, h].tolist())
+
+
+SMALL = [
+    # B, Hq, Hkv, lens, k, page_order
+    (1, 4, 4, [777], [9], "shuffled"),                      # G = 1
+    (2, 8, 4, [300, 1], [17, 1], "shuffled"),               # G = 2, N = 1
+    (3, 8, 2, [1000, 5000, 37], [20, 700, 37], "shuffled"),  # ragged tails; k == N
+    (2, 28, 4, [2500, 1999], [50, 40], "shuffled"),         # G = 7 (Qwen2.5-7B heads)
+    (2, 64, 8, [4096, 3000], [82, 60], "identity"),         # G = 8
+    (2, 32, 2, [3333, 1500], [67, 30], "shuffled"),         # G = 16
+    (4, 8, 2, [0, 15, 16, 17], [3, 20, 1, 5], "shuffled"),  # empty context, k > N, N < 16
+    (1, 8, 1, [20000], [1], "shuffled"),                    # k = 1
+    (1, 8, 2, [9000], [9000 // 3], "shuffled"),             # dense-ish selection (k = N/3)
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,lens,k,order", SMALL)
+def test_small_shapes(B, Hq, Hkv, lens, k, order):
+    w_cpu = wl.make_workload(B, Hq, Hkv, lens, k, seed=sum(lens) + Hq, page_order=order)
+    _run_small(w_cpu)
+
+
+def test_decode_on_oracle_indices():
+    """Feeds the oracle's own index sets to the GPU decode: isolates the decode kernel."""
+    w_cpu = wl.make_workload(2, 16, 4, [6000, 4100], [120, 90], seed=3)
+    w = w_cpu.to(DEV)
+    r = gh.Runner(w)
+    idx = oracle.topk(w_cpu.shape(), w_cpu.q, w_cpu.K, w_cpu.page_table, w_cpu.lens, w_cpu.k)
+    out = r.sparse(torch.from_numpy(idx).to(DEV))
+    assert r.device_status() == 0
+    ref = oracle.attend(w_cpu.shape(), w_cpu.q, w_cpu.K, w_cpu.V, w_cpu.page_table, w_cpu.lens, idx)
+    gh.check_outputs(out.cpu().numpy(), ref)
+
+
+def test_decode_arbitrary_index_sets():
+    """Per-head random subsets (no relation to the scores), different sizes per head, -1 padding."""
+    w_cpu = wl.make_workload(2, 16, 2, [5000, 3000], 1, seed=4, k_max=400)
+    g = torch.Generator().manual_seed(5)
+    idx = torch.full((2, 16, 400), -1, dtype=torch.int32)
+    for b in range(2):
+        for h in range(16):
+            cnt = int(torch.randint(0, 401, (1,), generator=g))
+            cnt = min(cnt, int(w_cpu.lens[b]))
+            sel = torch.randperm(int(w_cpu.lens[b]), generator=g)[:cnt].sort().values
+            idx[b, h, :cnt] = sel.to(torch.int32)
+    w = w_cpu.to(DEV)
+    r = gh.Runner(w)
+    out = r.sparse(idx.to(DEV))
+    assert r.device_status() == 0
+    ref = oracle.attend(w_cpu.shape(), w_cpu.q, w_cpu.K, w_cpu.V, w_cpu.page_table, w_cpu.lens, idx)
+    gh.check_outputs(out.cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("n,k", [(3000, 100), (40000, 100), (40000, 39999)])
+def test_exact_ties_go_to_lower_positions(n, k):
+    """Identical K rows: every score ties, so the selection is exactly positions 0..k-1.  With N
+    large the tied bin overflows the shared-memory candidate list (streaming refinement path)."""
+    w_cpu = wl.make_workload(1, 4, 1, n, k, seed=7)
+    w_cpu.K[:] = w_cpu.K[0, 0, 0]
+    w = w_cpu.to(DEV)
+    r = gh.Runner(w)
+    idx = r.topk().cpu().numpy()
+    assert r.device_status() == 0
+    assert (idx[0, :, :k] == np.arange(k)).all()
+    assert (idx[0, :, k:] == -1).all()
+
+
+def test_zero_scores_are_ties():
+    """K = 0 gives +0/-0 scores, which compare equal: the lowest positions win."""
+    w_cpu = wl.make_workload(1, 4, 2, 2000, 10, seed=8)
+    w_cpu.K.zero_()
+    w_cpu.q[0, 1] = -w_cpu.q[0, 1].abs()
+    w = w_cpu.to(DEV)
+    r = gh.Runner(w)
+    idx = r.topk().cpu().numpy()
+    assert r.device_status() == 0
+    assert (idx[0, :, :10] == np.arange(10)).all()
+
+
+def test_deterministic_and_placement_invariant():
+    """Two runs are bit-identical; moving pages to other physical slots changes nothing."""
+    w_cpu = wl.make_workload(2, 16, 4, [7000, 5000], [140, 100], seed=9, page_order="identity")
+    w = w_cpu.to(DEV)
+    r = gh.Runner(w)
+    i1, o1 = r.topk(), None
+    o1 = r.sparse(i1)
+    d1 = r.dense()
+    i2 = r.topk()
+    o2 = r.sparse(i2)
+    assert torch.equal(i1, i2) and torch.equal(o1, o2)
+    perm = torch.randperm(w_cpu.num_pages, generator=torch.Generator().manual_seed(1))
+    w2 = w_cpu.to("cpu")
+    K2 = torch.empty_like(w2.K)
+    V2 = torch.empty_like(w2.V)
+    K2[perm] = w2.K
+    V2[perm] = w2.V
+    pt2 = w2.page_table.clone()
+    valid = pt2 >= 0
+    pt2[valid] = perm[pt2[valid].long()].to(torch.int32)
+    w2.K, w2.V, w2.page_table = K2, V2, pt2
+    r2 = gh.Runner(w2.to(DEV))
+    i3 = r2.topk()
+    o3 = r2.sparse(i3)
+    d3 = r2.dense()
+    assert r.device_status() == 0 and r2.device_status() == 0
+    assert torch.equal(i1, i3) and torch.equal(o1, o3) and torch.equal(d1, d3)
+
+
+def test_llama8b_full():
+    w_cpu = wl.named("llama8b")
+    _run_small(w_cpu, check_dense=True)
+
+
+def _big(name, **kw):
+    torch.cuda.empty_cache()
+    w = wl.named(name, device=DEV, **kw)
+    return w, gh.Runner(w)
+
+
+def test_long128k_sampled():
+    w, r = _big("long128k")
+    idx = r.topk()
+    out = r.sparse(idx)
+    dense = r.dense()
+    assert r.device_status() == 0
+    gh.sampled_parity(w, idx, out, [(0, 0), (1, 3), (2, 5), (3, 7)], dense=dense)
+    # attention sinks: K rows 0-3 are scaled by 3, so a head whose q is aligned with them keeps them;
+    # at least the index rows must all be full
+    assert (idx[:, :, :2621] >= 0).all()
+
+
+@pytest.mark.parametrize("ratio", [10, 50, 100, 1])
+def test_sweep128k_sampled(ratio):
+    w, r = _big("sweep128k", ratio=ratio)
+    idx = r.topk()
+    out = r.sparse(idx)
+    dense = r.dense() if ratio == 1 else None
+    assert r.device_status() == 0
+    gh.sampled_parity(w, idx, out, [(0, 0), (15, 7)], dense=dense)
+    if ratio == 1:
+        assert torch.equal(out, dense)   # k = N: the sparse kernel reads every row, same arithmetic
+
+
+def test_ragged_steps_with_append():
+    w, r = _big("ragged")
+    steps = w.meta["steps"]
+    ratio = w.meta["ratio"]
+    checks = {0, steps // 2, steps - 1}
+    for t in range(steps):
+        w.q = w.meta["q_steps"][t].contiguous()
+        sdb.sd_append_kv(r.shape, w.K, w.V, w.page_table, w.lens, w.meta["k_new"][t], w.meta["v_new"][t], w.k, ratio,
+                         r.status)
+        idx = r.topk()
+        out = r.sparse(idx)
+        if t in checks:
+            assert r.device_status() == 0
+            lens = w.lens.cpu()
+            assert int(w.k[0]) == wl.k_for_ratio(int(lens[0]), ratio)
+            gh.sampled_parity(w, idx, out, [(0, 0), (int(torch.argmax(lens)), 3), (int(torch.argmin(lens)), 6)])
+    assert r.device_status() == 0
+
+
+# ----------------------------------------------------------------------------------------------
+# device-side error reporting (every bad value below is caught by the kernels' own checks)
+# ----------------------------------------------------------------------------------------------
+
+def _err_setup():
+    w_cpu = wl.make_workload(2, 8, 2, [500, 300], [10, 10], seed=11)
+    return w_cpu.to(DEV)
+
+
+def test_index_out_of_range_is_reported():
+    w = _err_setup()
+    r = gh.Runner(w)
+    idx = r.topk()
+    assert r.device_status() == 0
+    idx[1, 3, 9] = 400          # >= N_1 = 300, still ascending
+    r.sparse(idx)
+    assert r.device_status() == sdb.SD_ERR_INDEX_OOB
+
+
+def test_unsorted_indices_are_reported():
+    w = _err_setup()
+    r = gh.Runner(w)
+    idx = r.topk()
+    row = idx[0, 2, :10].flip(0).clone()
+    idx[0, 2, :10] = row
+    r.sparse(idx)
+    assert r.device_status() == sdb.SD_ERR_ORDER
+
+
+def test_bad_page_entry_is_reported():
+    w = _err_setup()
+    w.page_table[0, 3] = w.num_pages + 10
+    r = gh.Runner(w)
+    r.topk()
+    assert r.device_status() == sdb.SD_ERR_INDEX_OOB
+    r.status.zero_()
+    r.dense()
+    assert r.device_status() == sdb.SD_ERR_INDEX_OOB
+
+
+def test_bad_k_and_length_are_reported():
+    w = _err_setup()
+    r = gh.Runner(w)
+    k = torch.tensor([0, 10], dtype=torch.int32, device=DEV)
+    idx = r.topk(k=k)
+    assert r.device_status() == sdb.SD_ERR_INVALID_ARG
+    assert (idx[0] == -1).all()
+    r.status.zero_()
+    w.lens[1] = w.max_pages * w.P + 1
+    r.dense()
+    assert r.device_status() == sdb.SD_ERR_INVALID_ARG
