@@ -59,8 +59,8 @@ def source_hash(*names):
 
 
 KERNEL_SOURCES = {
-    "score_pass_kernel": ("topk_index.cu", "common.cuh"),
-    "select_kernel": ("topk_index.cu", "common.cuh"),
+    "score_pass_kernel": ("topk_score.cu", "common.cuh"),
+    "select_kernel": ("topk_select.cu", "common.cuh"),
     "decode_kernel": ("sparse_decode.cu", "common.cuh"),
 }
 
@@ -87,8 +87,11 @@ class ClockSampler:
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, device: int):
-        self.bus = torch.cuda.get_device_properties(device).pci_bus_id.lower() if hasattr(
-            torch.cuda.get_device_properties(device), "pci_bus_id") else None
+        props = torch.cuda.get_device_properties(device)
+        try:   # nvidia-smi prints the PCI id as DDDDDDDD:BB:DD.F
+            self.bus = f"{int(props.pci_bus_id):02x}:{int(props.pci_device_id):02x}.0"
+        except (AttributeError, TypeError, ValueError):
+            self.bus = None
         self.proc = None
         self.file = None
 
@@ -115,7 +118,7 @@ class ClockSampler:
         rows = [r.strip().split(", ") for r in self.file.read().splitlines() if r.strip()]
         os.unlink(self.file.name)
         if self.bus:
-            mine = [r for r in rows if r and r[0].lower().endswith(self.bus[-12:])]
+            mine = [r for r in rows if r and r[0].lower().endswith(self.bus)]
             rows = mine or rows
         sm, smax, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
@@ -219,12 +222,24 @@ def barrier(world):
 
 
 def max_over_ranks(world, x: float) -> float:
+    """Max of a per-rank scalar (a time) over all ranks; the only collective, measurement only."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(workload: str, rank: int) -> int:
+    """Each rank decodes its own batch: same shapes, different seeded data."""
+    return 1234 + wl.CONFIG_IDS[workload] + 1000 * rank
+
+
+def job_tokens_per_s(world: int, batch: int, ms_per_step_max: float) -> float:
+    """Whole-job throughput: every rank's batch, over the slowest rank's step time."""
+    return world * batch / (ms_per_step_max / 1e3)
 
 
 def config_of(w, args, world):
@@ -284,7 +299,7 @@ def run_ours(args):
     world, rank, local = dist_setup()
     dev = torch.device("cuda", local)
     kw = {"ratio": args.ratio} if args.workload == "sweep128k" else {}
-    w = wl.named(args.workload, device=dev, seed=1234 + wl.CONFIG_IDS[args.workload] + 1000 * rank, **kw)
+    w = wl.named(args.workload, device=dev, seed=rank_seed(args.workload, rank), **kw)
     shape = sdb.shape_of(w)
     ws_topk = sdb.workspace_for(shape, sdb.SD_OP_TOPK, dev)
     ws_dec = sdb.workspace_for(shape, sdb.SD_OP_SPARSE, dev)
@@ -379,7 +394,7 @@ def run_ours(args):
         return
     hbm, peak_kind = peaks()
     tokens = w.B * world
-    value = tokens / (t_step_max / 1e3)
+    value = job_tokens_per_s(world, w.B, t_step_max)
 
     def gbs(nbytes, ms):
         return nbytes / (ms / 1e3) / 1e9

@@ -19,7 +19,7 @@ constexpr int kSelectCapMax = 24 * 1024;      // select: candidate entries kept 
 struct DeviceInfo {
     bool ready = false;
     int sms = 0;
-    int decode_ctas_per_sm = 0;
+    int decode_ctas_per_sm[2][2] = {{0, 0}, {0, 0}};   // [dense][G > 8]
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -31,11 +31,15 @@ sd_status device_info(DeviceInfo* out) {
     std::lock_guard<std::mutex> lock(g_mu);
     DeviceInfo& d = g_dev[dev];
     if (!d.ready) {
-        int sms = 0, ctas = 0;
+        int sms = 0;
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return SD_ERR_CUDA;
-        if (decode_occupancy(&ctas) != cudaSuccess || ctas < 1) return SD_ERR_CUDA;
+        for (int dense = 0; dense < 2; ++dense)
+            for (int wide = 0; wide < 2; ++wide) {
+                int ctas = 0;
+                if (decode_occupancy(dense != 0, wide ? 16 : 8, &ctas) != cudaSuccess || ctas < 1) return SD_ERR_CUDA;
+                d.decode_ctas_per_sm[dense][wide] = ctas;
+            }
         d.sms = sms;
-        d.decode_ctas_per_sm = ctas;
         d.ready = true;
     }
     *out = d;
@@ -45,7 +49,8 @@ sd_status device_info(DeviceInfo* out) {
 struct Dims {
     int B, Hq, Hkv, G, max_pages, k_max, num_pages;
     long n_cap;   // max_pages * page size
-    int n_gran;   // 128-position granules of n_cap
+    int nr;       // union-building ranges per (b, kv head) group
+    int nrt;      // B * Hkv * nr
     int jmax;     // decode segment slots per (b, h)
 };
 
@@ -61,6 +66,9 @@ sd_status check_shape(const sd_shape* s, Dims* d) {
     const long n_cap = (long)s->max_pages_per_req * kPageSize;
     if (n_cap > (1L << 30)) return SD_ERR_UNSUPPORTED;
     if ((long)s->num_pages * kPageSize * s->num_kv_heads >= (1L << 32)) return SD_ERR_UNSUPPORTED;   // row index is 32-bit
+    const long nr = (n_cap + kRange - 1) / kRange;
+    const long nrt = (long)s->batch * s->num_kv_heads * nr;
+    if (nrt > kMaxRanges || nrt * kRange >= (1L << 31)) return SD_ERR_UNSUPPORTED;   // union rows are counted in int32
     d->B = s->batch;
     d->Hq = s->num_q_heads;
     d->Hkv = s->num_kv_heads;
@@ -69,8 +77,9 @@ sd_status check_shape(const sd_shape* s, Dims* d) {
     d->k_max = s->k_max;
     d->num_pages = s->num_pages;
     d->n_cap = n_cap;
-    d->n_gran = (int)((n_cap + 127) / 128);
-    d->jmax = d->n_gran + 1;
+    d->nr = (int)nr;
+    d->nrt = (int)nrt;
+    d->jmax = (int)((n_cap < kMaxDecodeWarps ? n_cap : kMaxDecodeWarps) + 1);
     return SD_OK;
 }
 
@@ -78,9 +87,26 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 size_t topk_workspace(const Dims& d) { return align256((size_t)d.B * d.Hq * d.n_cap * sizeof(float)); }
 
-// decode workspace: acc [B][Hq][jmax][128] fp32, then ml [B][Hq][jmax] float2
-size_t decode_acc_bytes(const Dims& d) { return align256((size_t)d.B * d.Hq * d.jmax * kHeadDim * sizeof(float)); }
-size_t decode_workspace(const Dims& d) { return decode_acc_bytes(d) + align256((size_t)d.B * d.Hq * d.jmax * sizeof(float2)); }
+// decode workspace, in order: acc [B][Hq][jmax][128] fp32, ml [B][Hq][jmax] float2,
+// bounds [B][Hq][nr + 1], entries [nrt][kRange] uint2, counts [nrt], offsets [nrt + 1], warp starts [kMaxDecodeWarps] int2, hdr [4]
+struct DecodeLayout {
+    size_t acc, ml, bounds, entries, counts, offsets, starts, hdr, total;
+};
+DecodeLayout decode_layout(const Dims& d) {
+    DecodeLayout L;
+    const size_t slots = (size_t)d.B * d.Hq * d.jmax;
+    L.acc = 0;
+    L.ml = L.acc + align256(slots * kHeadDim * sizeof(float));
+    L.bounds = L.ml + align256(slots * sizeof(float2));
+    L.entries = L.bounds + align256((size_t)d.B * d.Hq * (d.nr + 1) * sizeof(int));
+    L.counts = L.entries + align256((size_t)d.nrt * kRange * sizeof(uint2));
+    L.offsets = L.counts + align256((size_t)d.nrt * sizeof(int));
+    L.starts = L.offsets + align256(((size_t)d.nrt + 1) * sizeof(int));
+    L.hdr = L.starts + align256((size_t)kMaxDecodeWarps * sizeof(int2));
+    L.total = L.hdr + align256(4 * sizeof(int));
+    return L;
+}
+size_t decode_workspace(const Dims& d) { return decode_layout(d).total; }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -102,6 +128,8 @@ sd_status decode_common(const sd_shape* shape, const void* q, const void* K, con
     st = device_info(&di);
     if (st != SD_OK) return st;
     DecodeArgs a;
+    const DecodeLayout L = decode_layout(d);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
     a.q = static_cast<const __nv_bfloat16*>(q);
     a.K = static_cast<const __nv_bfloat16*>(K);
     a.V = static_cast<const __nv_bfloat16*>(V);
@@ -109,8 +137,14 @@ sd_status decode_common(const sd_shape* shape, const void* q, const void* K, con
     a.lens = lens;
     a.idx = dense ? nullptr : idx;
     a.out = out;
-    a.acc = static_cast<float*>(workspace);
-    a.ml = reinterpret_cast<float2*>(static_cast<uint8_t*>(workspace) + decode_acc_bytes(d));
+    a.acc = reinterpret_cast<float*>(ws + L.acc);
+    a.ml = reinterpret_cast<float2*>(ws + L.ml);
+    a.bounds = reinterpret_cast<int*>(ws + L.bounds);
+    a.entries = reinterpret_cast<uint2*>(ws + L.entries);
+    a.counts = reinterpret_cast<int*>(ws + L.counts);
+    a.offsets = reinterpret_cast<int*>(ws + L.offsets);
+    a.warp_start = reinterpret_cast<int2*>(ws + L.starts);
+    a.hdr = reinterpret_cast<int*>(ws + L.hdr);
     a.status = dev_status;
     a.B = d.B;
     a.Hq = d.Hq;
@@ -120,12 +154,22 @@ sd_status decode_common(const sd_shape* shape, const void* q, const void* K, con
     a.num_pages = d.num_pages;
     a.k_max = dense ? 0 : d.k_max;
     a.n_cap = d.n_cap;
+    a.nr = d.nr;
+    a.nrt = d.nrt;
     a.jmax = d.jmax;
-    const int ctas = di.sms * di.decode_ctas_per_sm;
-    a.total_warps = ctas * kDecodeWarpsPerCta;
+    int warps = di.sms * di.decode_ctas_per_sm[dense ? 1 : 0][d.G > 8 ? 1 : 0];
+    if (warps > kMaxDecodeWarps) warps = kMaxDecodeWarps;
+    a.total_warps = warps;   // one warp per CTA
     a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)kHeadDim));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    st = launch_status(launch_decode(a, dense, ctas, s));
+    if (cudaMemsetAsync(a.hdr + 2, 0, sizeof(int), s) != cudaSuccess) return SD_ERR_CUDA;   // union-pass ticket
+    if (!dense) {
+        st = launch_status(launch_bounds(a, s));
+        if (st != SD_OK) return st;
+    }
+    st = launch_status(launch_union(a, dense, s));
+    if (st != SD_OK) return st;
+    st = launch_status(launch_decode(a, dense, s));
     if (st != SD_OK) return st;
     return launch_status(launch_merge(a, s));
 }

@@ -98,6 +98,29 @@ def test_exact_ties_go_to_lower_positions(n, k):
     assert (idx[0, :, k:] == -1).all()
 
 
+def test_sampled_threshold_misplaced_falls_back():
+    """Every 32nd position scores high and all others score exactly 0.  The selector's strided sample
+    sees only the high positions, so its candidate threshold admits fewer rows than k; the exact
+    fallback must still return the 2048 high rows plus the lowest-position zeros."""
+    n, k = 65536, 3000
+    w_cpu = wl.make_workload(1, 1, 1, n, k, seed=12, page_order="shuffled")
+    q = w_cpu.q[0, 0]
+    high = torch.zeros(n, dtype=torch.bool)
+    high[::32] = True
+    pos = torch.arange(n)
+    pages = w_cpu.page_table[0].long()[pos // w_cpu.P]
+    slots = pos % w_cpu.P
+    K = w_cpu.K
+    K[pages, slots, 0] = 0
+    K[pages[high], slots[high], 0] = q
+    w = w_cpu.to(DEV)
+    r = gh.Runner(w)
+    idx = r.topk().cpu().numpy()
+    assert r.device_status() == 0
+    expect = sorted(set(range(0, n, 32)) | set([p for p in range(n) if p % 32][: k - 2048]))
+    assert idx[0, 0, :k].tolist() == expect
+
+
 def test_zero_scores_are_ties():
     """K = 0 gives +0/-0 scores, which compare equal: the lowest positions win."""
     w_cpu = wl.make_workload(1, 4, 2, 2000, 10, seed=8)
