@@ -111,6 +111,23 @@ SD_API sd_status sd_topk_scores(const sd_shape* shape, const void* q, const void
 SD_API sd_status sd_topk_select(const sd_shape* shape, const int32_t* lens, const int32_t* k, int32_t* idx,
                          void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream);
 
+/* sd_topk_index without a caller-provided workspace, for callers that cannot allocate device memory
+ * (for example a plugin inside a host engine that passes it only inputs and outputs, or a service
+ * whose device memory is fixed at start-up).  The pages have no counterpart of this entry point.
+ *   Same inputs, outputs, checks and results as sd_topk_index.  The fp32 scores live in one
+ *   file-scope device array of 32 MiB inside the library, held by every GPU that loads the library
+ *   until the process exits; the call allocates nothing.
+ *   Limit: B * Hq * max_pages_per_req * 16 scores must fit in 32 MiB (8,388,608 floats), else
+ *   SD_ERR_WORKSPACE and nothing is launched.
+ *   The first call on a device looks up the array's device address (cudaGetSymbolAddress) with that
+ *   device current; make that first call before any stream capture.
+ *   Every call on a device uses the same array, which keeps the last call's scores: calls whose
+ *   kernels overlap on the GPU (other streams, other host threads) race and must be serialised by
+ *   the caller. */
+SD_API sd_status sd_topk_index_static(const sd_shape* shape, const void* q, const void* K,
+                                      const int32_t* page_table, const int32_t* lens, const int32_t* k,
+                                      int32_t* idx, int32_t* dev_status, void* stream);
+
 /* Sparse decode attention over the selected rows ("Sparse" mode of Fig. 1(a) of "Inference-time
  * context sparsity"; SDPA of the xllm survey sec. 1.1 restricted to the selected set).
  *   out[b,h] = sum_{i in S} w_i V[b, h/G, i],  w = softmax over S of (q[b,h] . K[b,h/G,i]) / sqrt(d),

@@ -28,8 +28,8 @@ SD_OP_TOPK = 1
 SD_OP_SPARSE = 2
 SD_OP_DENSE = 3
 
-EXPORTED = ("sd_workspace_size", "sd_topk_index", "sd_topk_scores", "sd_topk_select", "sd_sparse_decode",
-            "sd_dense_decode", "sd_append_kv", "sd_status_string", "sd_version")
+EXPORTED = ("sd_workspace_size", "sd_topk_index", "sd_topk_scores", "sd_topk_select", "sd_topk_index_static",
+            "sd_sparse_decode", "sd_dense_decode", "sd_append_kv", "sd_status_string", "sd_version")
 
 
 class SdShape(ctypes.Structure):
@@ -63,6 +63,8 @@ def load():
     lib.sd_topk_index.argtypes = [SH, P, P, P, P, P, P, P, SZ, P, P]
     lib.sd_topk_scores.argtypes = [SH, P, P, P, P, P, P, SZ, P, P]
     lib.sd_topk_select.argtypes = [SH, P, P, P, P, SZ, P, P]
+    lib.sd_topk_index_static.argtypes = [SH, P, P, P, P, P, P, P, P]
+    lib.sd_topk_index_static.restype = I32
     lib.sd_sparse_decode.argtypes = [SH, P, P, P, P, P, P, P, P, SZ, P, P]
     lib.sd_dense_decode.argtypes = [SH, P, P, P, P, P, P, P, SZ, P, P]
     lib.sd_append_kv.argtypes = [SH, P, P, P, P, P, P, P, I32, P, P]
@@ -143,6 +145,13 @@ def sd_topk_select(shape, lens, k, idx, workspace, dev_status, stream=None, chec
     st = load().sd_topk_select(ctypes.byref(shape), _ptr(lens), _ptr(k), _ptr(idx), _ptr(workspace),
                                _ws_bytes(workspace), _ptr(dev_status), _stream(stream))
     return _check(st, "sd_topk_select", check)
+
+
+def sd_topk_index_static(shape, q, K, page_table, lens, k, idx, dev_status, stream=None, check=True) -> int:
+    """sd_topk_index with the library's own static 32 MiB score scratch (no workspace argument)."""
+    st = load().sd_topk_index_static(ctypes.byref(shape), _ptr(q), _ptr(K), _ptr(page_table), _ptr(lens), _ptr(k),
+                                     _ptr(idx), _ptr(dev_status), _stream(stream))
+    return _check(st, "sd_topk_index_static", check)
 
 
 def sd_sparse_decode(shape, q, K, V, page_table, lens, idx, out, workspace, dev_status, stream=None,
