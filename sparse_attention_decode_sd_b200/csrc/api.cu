@@ -68,7 +68,7 @@ sd_status check_shape(const sd_shape* s, Dims* d) {
     if ((long)s->num_pages * kPageSize * s->num_kv_heads >= (1L << 32)) return SD_ERR_UNSUPPORTED;   // row index is 32-bit
     const long nr = (n_cap + kRange - 1) / kRange;
     const long nrt = (long)s->batch * s->num_kv_heads * nr;
-    if (nrt > kMaxRanges || nrt * kRange >= (1L << 31)) return SD_ERR_UNSUPPORTED;   // union rows are counted in int32
+    if (nrt * kRange >= (1L << 31)) return SD_ERR_UNSUPPORTED;   // union rows are counted in int32
     d->B = s->batch;
     d->Hq = s->num_q_heads;
     d->Hkv = s->num_kv_heads;
@@ -88,22 +88,19 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 size_t topk_workspace(const Dims& d) { return align256((size_t)d.B * d.Hq * d.n_cap * sizeof(float)); }
 
 // decode workspace, in order: acc [B][Hq][jmax][128] fp32, ml [B][Hq][jmax] float2,
-// bounds [B][Hq][nr + 1], entries [nrt][kRange] uint2, counts [nrt], offsets [nrt + 1], warp starts [kMaxDecodeWarps] int2, hdr [4]
+// entries [nrt][kRange] uint2, counts [nrt], hdr [4] followed by per-group totals [B * Hkv]
 struct DecodeLayout {
-    size_t acc, ml, bounds, entries, counts, offsets, starts, hdr, total;
+    size_t acc, ml, entries, counts, hdr, total;
 };
 DecodeLayout decode_layout(const Dims& d) {
     DecodeLayout L;
     const size_t slots = (size_t)d.B * d.Hq * d.jmax;
     L.acc = 0;
     L.ml = L.acc + align256(slots * kHeadDim * sizeof(float));
-    L.bounds = L.ml + align256(slots * sizeof(float2));
-    L.entries = L.bounds + align256((size_t)d.B * d.Hq * (d.nr + 1) * sizeof(int));
+    L.entries = L.ml + align256(slots * sizeof(float2));
     L.counts = L.entries + align256((size_t)d.nrt * kRange * sizeof(uint2));
-    L.offsets = L.counts + align256((size_t)d.nrt * sizeof(int));
-    L.starts = L.offsets + align256(((size_t)d.nrt + 1) * sizeof(int));
-    L.hdr = L.starts + align256((size_t)kMaxDecodeWarps * sizeof(int2));
-    L.total = L.hdr + align256(4 * sizeof(int));
+    L.hdr = L.counts + align256((size_t)d.nrt * sizeof(int));
+    L.total = L.hdr + align256((4 + (size_t)d.B * d.Hkv) * sizeof(int));
     return L;
 }
 size_t decode_workspace(const Dims& d) { return decode_layout(d).total; }
@@ -139,12 +136,10 @@ sd_status decode_common(const sd_shape* shape, const void* q, const void* K, con
     a.out = out;
     a.acc = reinterpret_cast<float*>(ws + L.acc);
     a.ml = reinterpret_cast<float2*>(ws + L.ml);
-    a.bounds = reinterpret_cast<int*>(ws + L.bounds);
     a.entries = reinterpret_cast<uint2*>(ws + L.entries);
     a.counts = reinterpret_cast<int*>(ws + L.counts);
-    a.offsets = reinterpret_cast<int*>(ws + L.offsets);
-    a.warp_start = reinterpret_cast<int2*>(ws + L.starts);
     a.hdr = reinterpret_cast<int*>(ws + L.hdr);
+    a.gtot = a.hdr + 4;
     a.status = dev_status;
     a.B = d.B;
     a.Hq = d.Hq;
@@ -162,11 +157,8 @@ sd_status decode_common(const sd_shape* shape, const void* q, const void* K, con
     a.total_warps = warps;   // one warp per CTA
     a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)kHeadDim));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (cudaMemsetAsync(a.hdr + 2, 0, sizeof(int), s) != cudaSuccess) return SD_ERR_CUDA;   // union-pass ticket
-    if (!dense) {
-        st = launch_status(launch_bounds(a, s));
-        if (st != SD_OK) return st;
-    }
+    st = launch_status(launch_prep(a, s));   // zero the row totals the union pass accumulates
+    if (st != SD_OK) return st;
     st = launch_status(launch_union(a, dense, s));
     if (st != SD_OK) return st;
     st = launch_status(launch_decode(a, dense, s));

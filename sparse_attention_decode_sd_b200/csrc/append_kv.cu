@@ -6,6 +6,7 @@
 namespace sd {
 
 __global__ void __launch_bounds__(128) append_kernel(AppendArgs a) {
+    pdl_enter();
     const int b = blockIdx.x;
     __shared__ long s_row;
     __shared__ int s_ok;
@@ -44,8 +45,8 @@ __global__ void __launch_bounds__(128) append_kernel(AppendArgs a) {
 }
 
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t stream) {
-    append_kernel<<<a.B, 128, 0, stream>>>(a);
-    return cudaGetLastError();
+    cudaError_t e = launch_pdl(append_kernel, dim3(a.B), dim3(128), 0, stream, a);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace sd

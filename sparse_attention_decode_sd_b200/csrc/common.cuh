@@ -167,6 +167,33 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* scratch, int* to
     return res;
 }
 
+// ---------------------------------------------------------------------------------------------
+// Programmatic dependent launch.  Every kernel of the library is launched so that its launch may
+// overlap the tail of the kernel before it in the stream: it first lets its own dependants launch,
+// then waits until the previous kernel has completed and its memory is visible, before touching
+// anything.  (Both instructions are no-ops when a kernel was launched without the attribute.)
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_enter() {
+    asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+    asm volatile("griddepcontrol.wait;\n" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // Request lengths validated on the device: an invalid length is reported and treated as 0.
 __device__ __forceinline__ int checked_len(const int32_t* lens, int b, long n_cap, int32_t* status) {
     const int n = lens[b];

@@ -31,7 +31,6 @@ cudaError_t launch_select(const TopkArgs& a, cudaStream_t stream);
 
 constexpr int kRange = 8192;            // positions per union-building range
 constexpr int kMaxDecodeWarps = 1280;   // persistent decode warps (one per CTA) at most
-constexpr int kMaxRanges = 16384;       // B * Hkv * ranges per group at most
 
 struct DecodeArgs {
     const __nv_bfloat16* q;
@@ -42,12 +41,10 @@ struct DecodeArgs {
     const int32_t* idx;   // null for dense decode
     float* out;
     // workspace
-    int* bounds;          // [B * Hq][nr + 1]: first idx entry of each range, per (b, h) row
     uint2* entries;       // per range: union rows {cache row index, head mask}, ascending positions
     int* counts;          // [nrt] union rows per range
-    int* offsets;         // [nrt + 1] exclusive prefix of counts (offsets[nrt] = E)
-    int2* warp_start;     // [total_warps] first (range, offset) of each decode warp
-    int* hdr;             // [0] E, [1] rows per warp, [2] ticket of the union pass
+    int* hdr;             // [0] E = all union rows; followed by gtot[B * Hkv], union rows per group
+    int* gtot;            // = hdr + 4 (zeroed together with hdr before the union pass)
     float2* ml;           // per (b, h, segment) running max (log2 units) and sum
     float* acc;           // per (b, h, segment) un-normalised output [128]
     int32_t* status;
@@ -64,7 +61,7 @@ size_t decode_smem();
 size_t union_smem(const DecodeArgs& a);
 // CTAs (one warp each) of the decode kernel variant for (dense, G) that fit on one SM.
 cudaError_t decode_occupancy(bool dense, int G, int* ctas_per_sm);
-cudaError_t launch_bounds(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_prep(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_union(const DecodeArgs& a, bool dense, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs& a, bool dense, cudaStream_t stream);
 cudaError_t launch_merge(const DecodeArgs& a, cudaStream_t stream);

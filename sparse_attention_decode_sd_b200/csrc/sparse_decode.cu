@@ -4,17 +4,18 @@
 // ("Dense" mode of the same figure).
 //
 // Three kernels per call:
-//   union_kernel   one CTA per 8192-position range of each (request, KV head) group: marks which of
-//                  the group's G query heads selected each position, and writes the ascending union
-//                  of the group's selections as {cache row index (page table applied), head mask}.
-//                  The last CTA to finish prefix-sums the per-range counts and cuts the flattened
-//                  union-row sequence evenly across the decode warps.  (Dense decode: every
-//                  position is a row and no list is written.)
-//   decode_kernel  one warp per CTA, a persistent grid of one wave.  Each warp streams its share of
-//                  union rows in tiles of 16: every row is fetched once for all heads of its group
-//                  with 16-byte cp.async gathers (256-byte K and V rows into 272-byte padded
-//                  shared-memory rows, three tiles in flight).  On the
-//                  tensor cores (mma.sync m16n8k16, bf16 in, fp32 accumulate):
+//   union_kernel   one CTA per 8192-position range of each (request, KV head) group: finds each head's
+//                  slice of its idx row for the range (warp-cooperative search), marks which of the
+//                  group's G query heads selected each position, and writes the ascending union of
+//                  the group's selections as {cache row index (page table applied), head mask}; the
+//                  row counts are added atomically to per-group and global totals.  (Dense decode:
+//                  every position is a row and no list is written.)
+//   decode_kernel  one warp per CTA, a persistent grid of one wave.  The union rows of all groups,
+//                  in (request, KV head, position) order, are cut evenly across the warps; each warp
+//                  locates its start from the totals and streams its rows in tiles of 16: every row
+//                  is fetched once for all heads of its group with 16-byte cp.async gathers (256-byte
+//                  K and V rows into 272-byte padded shared-memory rows, three tiles in flight).  On
+//                  the tensor cores (mma.sync m16n8k16, bf16 in, fp32 accumulate):
 //                      S   = K_tile (16 rows x 128) . Q^T (128 x 8 heads)          8 MMAs / 8 heads
 //                      O^T += V_tile^T (128 x 16 rows) . P (16 rows x 8 heads)     16 MMAs / 8 heads
 //                  Heads that did not select a row get -inf before an fp32 online softmax; P goes to
@@ -38,49 +39,36 @@ constexpr int kFlagFirst = 1, kFlagLast = 2, kFlagEnd = 4;
 // ---------------------------------------------------------------------------------------------
 // union_kernel
 // ---------------------------------------------------------------------------------------------
-__device__ __forceinline__ int len_checked(const DecodeArgs& a, int b) {
-    return checked_len(a.lens, b, a.n_cap, a.status);
-}
-
 size_t union_smem(const DecodeArgs& a) {
-    const size_t build = sizeof(uint32_t) * (kRange / 2) + sizeof(int) * (kRange / kPageSize);
-    const size_t tail = sizeof(int) * ((size_t)a.nrt + 1);
-    return sizeof(int) * 64 + (build > tail ? build : tail);
+    (void)a;
+    return sizeof(int) * 64 + sizeof(uint32_t) * (kRange / 2) + sizeof(uint32_t) * (kRange / 32) +
+           sizeof(int) * (kRange / kPageSize);
 }
 
-// One thread per idx entry (grid: entry chunks x rows): entry i of row (b, h) opens every range r'
-// in (range(prev), range(v)] -- bounds[b,h][r'] = i -- and the row's last valid entry closes the
-// remaining ranges.  Every slot of a well-formed row is written exactly once, so nothing needs
-// clearing.  Also checks the row: entries must lie in [0, N_b) and be strictly ascending, with
-// padding only at the end.
-__global__ void __launch_bounds__(256) bounds_kernel(DecodeArgs a) {
-    const int lane = threadIdx.x & 31;
-    const long bh = blockIdx.y;
-    const int i = blockIdx.x * blockDim.x + threadIdx.x;
-    const int b = (int)(bh / a.Hq);
-    const int n = len_checked(a, b);
-    const int32_t* row = a.idx + bh * a.k_max;
-    const int v = (i < a.k_max) ? row[i] : -1;
-    int prev = __shfl_up_sync(0xffffffffu, v, 1);
-    int next = __shfl_down_sync(0xffffffffu, v, 1);
-    if (lane == 0) prev = (i > 0 && i - 1 < a.k_max) ? row[i - 1] : -1;
-    if (lane == 31 || i + 1 >= a.k_max) next = (i + 1 < a.k_max) ? row[i + 1] : -1;
-    if (i >= a.k_max) return;
-    int* bounds = a.bounds + bh * (a.nr + 1);
-    const bool valid = v >= 0 && v < n;
-    if (v >= n) report(a.status, SD_ERR_INDEX_OOB);
-    if (v >= 0 && i > 0 && (prev < 0 || prev >= v)) report(a.status, SD_ERR_ORDER);
-    const bool prev_valid = i > 0 && prev >= 0 && prev < n;
-    if (valid) {
-        const int rv = v / kRange;
-        const int rp = prev_valid ? min(prev / kRange, rv) : -1;
-        for (int r = rp + 1; r <= rv; ++r) bounds[r] = i;
-        const bool next_valid = next >= 0 && next < n;
-        if (!next_valid)
-            for (int r = rv + 1; r <= a.nr; ++r) bounds[r] = i + 1;
-    } else if (i == 0) {   // a row that starts with padding has no selected rows
-        for (int r = 0; r <= a.nr; ++r) bounds[r] = 0;
+// The slice [s, e) of an ascending, -1-padded row whose entries lie in [lo, hi): lanes 0..15 search
+// for the first entry >= lo, lanes 16..31 for the first entry >= hi (negative entries count as +inf),
+// 17-way per round.  Malformed rows still end the search in range.
+__device__ __forceinline__ int2 warp_slice(const int32_t* row, int len, int lo, int hi) {
+    const int lane = threadIdx.x & 31, half = lane >> 4, sub = lane & 15;
+    const int target = half ? hi : lo;
+    int l = 0, h = len;   // the answer lies in [l, h]
+    while (__any_sync(0xffffffffu, l < h)) {
+        const bool busy = l < h;
+        const int span = h - l;
+        const int p = l + (int)(((long)(sub + 1) * span) / 17);
+        const int v = busy ? __ldg(row + p) : 0;
+        const uint32_t bal = __ballot_sync(0xffffffffu, busy && v >= 0 && v < target);
+        const int cnt = __popc((bal >> (half * 16)) & 0xffffu);
+        if (busy) {
+            const int nl = cnt > 0 ? l + (int)(((long)cnt * span) / 17) + 1 : l;
+            const int nh = cnt < 16 ? l + (int)(((long)(cnt + 1) * span) / 17) : h;
+            l = nl;
+            h = nh;
+        }
     }
+    const int s = __shfl_sync(0xffffffffu, l, 0);
+    const int e = __shfl_sync(0xffffffffu, l, 16);
+    return make_int2(s, max(s, e));
 }
 
 template <bool DENSE>
@@ -88,10 +76,10 @@ __global__ void __launch_bounds__(kUnionThreads, 4) union_kernel(DecodeArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     int* scratch = reinterpret_cast<int*>(smem);                 // [64]
     uint32_t* mask = reinterpret_cast<uint32_t*>(scratch + 64);  // [kRange / 2]: two 16-bit head masks per word
-    int* pt = reinterpret_cast<int*>(mask + kRange / 2);         // [kRange / 16]
-    __shared__ int s_last;
-    __shared__ int s_lo[kMaxGroup], s_len[kMaxGroup], s_pre[kMaxGroup + 1];
-    const int tid = threadIdx.x;
+    uint32_t* any = mask + kRange / 2;                           // [kRange / 32]: 1 bit per selected position
+    int* pt = reinterpret_cast<int*>(any + kRange / 32);         // [kRange / 16]
+    pdl_enter();
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
     const int ri = blockIdx.x;
     const int grp = ri / a.nr, r = ri - grp * a.nr;
     const int b = grp / a.Hkv, kvh = grp - b * a.Hkv;
@@ -102,8 +90,8 @@ __global__ void __launch_bounds__(kUnionThreads, 4) union_kernel(DecodeArgs a) {
         if constexpr (DENSE) {
             cnt = hi - lo;
         } else {
-            uint4* m4 = reinterpret_cast<uint4*>(mask);
-            for (int i = tid; i < kRange / 8; i += blockDim.x) m4[i] = make_uint4(0, 0, 0, 0);
+            uint4* m4 = reinterpret_cast<uint4*>(mask);   // mask and any are contiguous
+            for (int i = tid; i < (kRange / 2 + kRange / 32) / 4; i += blockDim.x) m4[i] = make_uint4(0, 0, 0, 0);
             const int np = (hi - lo + kPageSize - 1) / kPageSize;
             const int32_t* ptrow = a.page_table + (long)b * a.max_pages + lo / kPageSize;
             for (int i = tid; i < np; i += blockDim.x) {
@@ -114,131 +102,71 @@ __global__ void __launch_bounds__(kUnionThreads, 4) union_kernel(DecodeArgs a) {
                 }
                 pt[i] = page;
             }
-            if (tid < a.G) {   // this range's slice [s, e) of each head's row (clamped: rows may be malformed)
-                const int* bd = a.bounds + ((long)b * a.Hq + (long)kvh * a.G + tid) * (a.nr + 1);
-                const int s = min(max(bd[r], 0), a.k_max);
-                const int e = min(max(bd[r + 1], s), a.k_max);
-                s_lo[tid] = s;
-                s_len[tid] = e - s;
-            }
             __syncthreads();
-            if (tid == 0) {
-                int acc = 0;
-                for (int g = 0; g < a.G; ++g) {
-                    s_pre[g] = acc;
-                    acc += s_len[g];
-                }
-                s_pre[a.G] = acc;
-            }
-            __syncthreads();
-            // every thread marks entries of the flattened slices, eight independent loads at a time
-            const int tot_e = s_pre[a.G];
-            const int32_t* rows0 = a.idx + ((long)b * a.Hq + (long)kvh * a.G) * a.k_max;
-            constexpr int kBatch = 8;
-            for (int x0 = 0; x0 < tot_e; x0 += kBatch * kUnionThreads) {
-                int v[kBatch], gg[kBatch];
+            for (int g = warp; g < a.G; g += nwarps) {
+                const int32_t* row = a.idx + ((long)b * a.Hq + (long)kvh * a.G + g) * a.k_max;
+                const int2 se = warp_slice(row, a.k_max, lo, hi);
+                // chunks of 32 entries, four chunks' loads in flight; each entry is checked against
+                // its predecessor in the row (strictly ascending, inside this range)
+                for (int i0 = se.x; i0 < se.y; i0 += 128) {
+                    int v[4], pv[4];
 #pragma unroll
-                for (int u = 0; u < kBatch; ++u) {
-                    const int x = x0 + u * kUnionThreads + tid;
-                    v[u] = -1;
-                    gg[u] = 0;
-                    if (x < tot_e) {
-                        int g = 0;
-                        while (x >= s_pre[g + 1]) ++g;
-                        gg[u] = g;
-                        v[u] = __ldg(rows0 + (long)g * a.k_max + s_lo[g] + (x - s_pre[g]));
+                    for (int u = 0; u < 4; ++u) {
+                        const int i = i0 + 32 * u + lane;
+                        v[u] = (i < se.y) ? __ldg(row + i) : -1;
+                        pv[u] = (lane == 0 && i < se.y && i > 0) ? __ldg(row + i - 1) : -1;
                     }
-                }
 #pragma unroll
-                for (int u = 0; u < kBatch; ++u)
-                    if (v[u] >= lo && v[u] < hi) {
-                        const int o = v[u] - lo;
-                        atomicOr(&mask[o >> 1], (1u << gg[u]) << ((o & 1) * 16));
-                    }
-            }
-            __syncthreads();
-            // ordered compaction: thread t owns positions [32t, 32t + 32) of the range
-            constexpr int kPer = kRange / kUnionThreads;
-            const int o0 = tid * kPer;
-            uint32_t words[kPer / 2];
-            int c = 0;
-#pragma unroll
-            for (int k = 0; k < kPer / 2; ++k) {
-                words[k] = mask[o0 / 2 + k];
-                const int o = o0 + 2 * k;
-                const bool v0 = o < hi - lo && (words[k] & 0xffffu) && pt[o >> 4] >= 0;
-                const bool v1 = o + 1 < hi - lo && (words[k] >> 16) && pt[o >> 4] >= 0;
-                c += v0 + v1;
-            }
-            int tot;
-            int w = block_exclusive_scan(c, scratch, &tot);
-            uint2* dst = a.entries + (long)ri * kRange;
-#pragma unroll
-            for (int k = 0; k < kPer / 2; ++k) {
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int o = o0 + 2 * k + h;
-                    const uint32_t m = (words[k] >> (16 * h)) & 0xffffu;
-                    if (o < hi - lo && m) {
-                        const int page = pt[o >> 4];
-                        if (page >= 0) {
-                            const int p = lo + o;
-                            const uint32_t rowi =
-                                ((uint32_t)page * kPageSize + (uint32_t)(p & (kPageSize - 1))) * (uint32_t)a.Hkv + kvh;
-                            dst[w++] = make_uint2(rowi, m);
+                    for (int u = 0; u < 4; ++u) {
+                        const int i = i0 + 32 * u + lane;
+                        int prev = __shfl_up_sync(0xffffffffu, v[u], 1);
+                        if (lane == 0) prev = pv[u];
+                        if (i < se.y) {
+                            if (v[u] < lo || v[u] >= hi || (prev >= 0 && prev >= v[u])) {
+                                report(a.status, SD_ERR_ORDER);
+                            } else {
+                                const int o = v[u] - lo;
+                                atomicOr(&mask[o >> 1], (1u << g) << ((o & 1) * 16));
+                                atomicOr(&any[o >> 5], 1u << (o & 31));
+                            }
                         }
                     }
+                }
+                // the last range of a request: every entry after it must be padding
+                if (hi == n && lane == 0 && se.y < a.k_max && __ldg(row + se.y) >= 0) report(a.status, SD_ERR_INDEX_OOB);
+            }
+            __syncthreads();
+            // ordered compaction: thread t owns the 32 positions of bitmap word t
+            static_assert(kRange / 32 == kUnionThreads, "one bitmap word per thread");
+            uint32_t word = any[tid];
+            const int o0 = tid * 32;
+            int tot;
+            int w = block_exclusive_scan(__popc(word), scratch, &tot);
+            uint2* dst = a.entries + (long)ri * kRange;
+            while (word) {
+                const int o = o0 + __ffs(word) - 1;
+                word &= word - 1u;
+                const int page = pt[o >> 4];
+                const uint32_t m = (mask[o >> 1] >> ((o & 1) * 16)) & 0xffffu;
+                if (page >= 0) {
+                    const int p = lo + o;
+                    const uint32_t rowi =
+                        ((uint32_t)page * kPageSize + (uint32_t)(p & (kPageSize - 1))) * (uint32_t)a.Hkv + kvh;
+                    dst[w++] = make_uint2(rowi, m);
+                } else {
+                    dst[w++] = make_uint2(0u, 0u);   // invalid page (reported): a row no head attends to
                 }
             }
             cnt = tot;
         }
     }
-    if (tid == 0) a.counts[ri] = cnt;
-
-    // The last CTA to finish: prefix over all ranges and the decode warps' starting points.
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) s_last = (atomicAdd(&a.hdr[2], 1) == (int)gridDim.x - 1);
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-    int* offs = scratch + 64;   // [nrt + 1]
-    const volatile int* vcounts = a.counts;
-    int carry = 0;
-    for (int base = 0; base < a.nrt; base += blockDim.x) {
-        const int i = base + tid;
-        const int v = (i < a.nrt) ? vcounts[i] : 0;
-        int tot;
-        const int ex = block_exclusive_scan(v, scratch, &tot);
-        if (i < a.nrt) {
-            offs[i] = carry + ex;
-            a.offsets[i] = carry + ex;
-        }
-        carry += tot;
-    }
-    const int E = carry;
-    const int epw = max(1, (int)(((long)E + a.total_warps - 1) / a.total_warps));
     if (tid == 0) {
-        offs[a.nrt] = E;
-        a.offsets[a.nrt] = E;
-        a.hdr[0] = E;
-        a.hdr[1] = epw;
-    }
-    __syncthreads();
-    for (int w = tid; w < a.total_warps; w += blockDim.x) {
-        const long e0 = (long)w * epw;
-        int2 start = make_int2(-1, 0);
-        if (e0 < E) {   // largest range with offs <= e0 (it is non-empty)
-            int l = 0, h = a.nrt;
-            while (h - l > 1) {
-                const int mid = (l + h) >> 1;
-                if (offs[mid] <= e0) l = mid; else h = mid;
-            }
-            start = make_int2(l, (int)(e0 - offs[l]));
+        a.counts[ri] = cnt;
+        if (cnt > 0) {
+            atomicAdd(&a.gtot[grp], cnt);
+            atomicAdd(&a.hdr[0], cnt);
         }
-        a.warp_start[w] = start;
     }
-    if (tid == 0) a.hdr[2] = 0;   // ticket ready for the next call
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -338,7 +266,7 @@ __device__ __forceinline__ TileDesc prefetch_tile(const DecodeArgs& a, Walker& w
             w.off = 0;
             w.cnt = c;
             w.grp = ri / a.nr;
-            w.seg_j = (int)(blockIdx.x - __ldg(a.offsets + w.grp * a.nr) / w.epw);
+            w.seg_j = (int)(blockIdx.x - w.e / w.epw);   // w.e is the first row of the new group
             w.seg_new = true;
         }
     }
@@ -462,9 +390,11 @@ __device__ __forceinline__ void compute_tile(const DecodeArgs& a, const DecodeSm
     const int mi = lane >> 3, r8 = lane & 7;
 
     // S (16 rows x 8 heads per nt) = K_tile . Q^T
-    float s[NT][4];
+    float s[NT][4], s2[NT][4];   // two accumulators (even / odd k-blocks) halve the MMA dependency chain
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s[nt][e] = s2[nt][e] = 0.f;
     {
         const uint32_t rowaddr = kbase + (uint32_t)((((mi & 1) << 3) + r8) * kRowPitch + ((mi >> 1) << 4));
 #pragma unroll
@@ -472,8 +402,15 @@ __device__ __forceinline__ void compute_tile(const DecodeArgs& a, const DecodeSm
             uint32_t a0, a1, a2, a3;
             ldmatrix_x4(rowaddr + 32 * j, a0, a1, a2, a3);
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(s[nt], a0, a1, a2, a3, st.qb[nt][j][0], st.qb[nt][j][1]);
+            for (int nt = 0; nt < NT; ++nt) {
+                if (j & 1) mma_bf16_16816(s2[nt], a0, a1, a2, a3, st.qb[nt][j][0], st.qb[nt][j][1]);
+                else mma_bf16_16816(s[nt], a0, a1, a2, a3, st.qb[nt][j][0], st.qb[nt][j][1]);
+            }
         }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) s[nt][e] += s2[nt][e];
     }
     // mask heads that did not select a row (rows g and g+8 of the tile), online softmax per head
     const uint32_t mr0 = ws.meta_mask[stage][g], mr1 = ws.meta_mask[stage][g + 8];
@@ -546,19 +483,60 @@ template <bool DENSE, int NT>
 __global__ void __launch_bounds__(32) decode_kernel(DecodeArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     DecodeSmem& ws = *reinterpret_cast<DecodeSmem*>(smem);
+    pdl_enter();
 
-    const int2 start = a.warp_start[blockIdx.x];
-    if (start.x < 0) return;
+    const int lane = threadIdx.x & 31;
     const int E = a.hdr[0];
+    if (E == 0) return;
     Walker w;
-    w.epw = a.hdr[1];
+    w.epw = max(1, (int)(((long)E + a.total_warps - 1) / a.total_warps));
     w.e = (int)blockIdx.x * w.epw;
+    if (w.e >= E) return;
     w.e_end = min(E, w.e + w.epw);
-    w.ri = start.x;
-    w.off = start.y;
+    // the group holding row w.e (prefix over the per-group totals), then its range
+    int e0grp = 0;
+    w.grp = -1;
+    {
+        const int ngroups = a.B * a.Hkv;
+        int acc = 0;
+        for (int base = 0; base < ngroups && w.grp < 0; base += 32) {
+            const int v = (base + lane < ngroups) ? __ldg(a.gtot + base + lane) : 0;
+            int incl = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int t = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += t;
+            }
+            const int tot = __shfl_sync(0xffffffffu, incl, 31);
+            if (w.e < acc + tot) {
+                const int l = __ffs(__ballot_sync(0xffffffffu, acc + incl > w.e)) - 1;
+                w.grp = base + l;
+                e0grp = acc + __shfl_sync(0xffffffffu, incl - v, l);
+            }
+            acc += tot;
+        }
+        const int off_g = w.e - e0grp;
+        int acc2 = 0;
+        w.ri = -1;
+        for (int base = 0; base < a.nr && w.ri < 0; base += 32) {
+            const int v = (base + lane < a.nr) ? __ldg(a.counts + w.grp * a.nr + base + lane) : 0;
+            int incl = v;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int t = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += t;
+            }
+            const int tot = __shfl_sync(0xffffffffu, incl, 31);
+            if (off_g < acc2 + tot) {
+                const int l = __ffs(__ballot_sync(0xffffffffu, acc2 + incl > off_g)) - 1;
+                w.ri = w.grp * a.nr + base + l;
+                w.off = off_g - (acc2 + __shfl_sync(0xffffffffu, incl - v, l));
+            }
+            acc2 += tot;
+        }
+    }
     w.cnt = __ldg(a.counts + w.ri);
-    w.grp = w.ri / a.nr;
-    w.seg_j = (int)(blockIdx.x - __ldg(a.offsets + w.grp * a.nr) / w.epw);
+    w.seg_j = (int)(blockIdx.x - e0grp / w.epw);
     w.seg_new = true;
 
     Softmax<NT> st;
@@ -571,13 +549,14 @@ __global__ void __launch_bounds__(32) decode_kernel(DecodeArgs a) {
     }
     for (int t = 0;; ++t) {
         const int stage = t % kStages;
-        cp_async_wait<kStages - 2>();
+        // the stage of tile t-1 is free: issue tile t+kStages-1 before waiting for tile t
+        issue_tile(a, ws, (t + kStages - 1) % kStages, next);
+        next = prefetch_tile<DENSE>(a, w);
+        cp_async_wait<kStages - 1>();
         __syncwarp();
         const int rows = ws.info[stage][0], flags = ws.info[stage][1];
         if (flags & kFlagEnd) break;
         const int tb = ws.info[stage][2], tkvh = ws.info[stage][3], tj = ws.info[stage][4];
-        issue_tile(a, ws, (t + kStages - 1) % kStages, next);
-        next = prefetch_tile<DENSE>(a, w);
         if (flags & kFlagFirst) load_q(a, tb, tkvh, st);
         if (rows > 0) compute_tile(a, ws, stage, st);
         if (flags & kFlagLast) {
@@ -595,12 +574,26 @@ __global__ void __launch_bounds__(kHeadDim) merge_kernel(DecodeArgs a) {
     __shared__ float s_m[32];   // per-segment weights of the current chunk
     __shared__ float s_l[32];
     __shared__ float s_scale[1];
+    pdl_enter();
     const int d = threadIdx.x;
     const long bh = blockIdx.x;
     const int b = (int)(bh / a.Hq), h = (int)(bh % a.Hq), kvh = h / a.G;
+    __shared__ int s_e0;
     const int grp = b * a.Hkv + kvh;
-    const int e0 = a.offsets[grp * a.nr], e1 = a.offsets[(grp + 1) * a.nr];
-    const int epw = a.hdr[1];
+    if (d < 32) {   // first union row of the group: prefix over the per-group totals
+        int acc = 0;
+        for (int base = 0; base < grp; base += 32) {
+            int v = (base + d < grp) ? a.gtot[base + d] : 0;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+            acc += v;
+        }
+        if (d == 0) s_e0 = acc;
+    }
+    __syncthreads();
+    const int E = a.hdr[0];
+    const int epw = max(1, (int)(((long)E + a.total_warps - 1) / a.total_warps));
+    const int e0 = s_e0, e1 = e0 + a.gtot[grp];
     const int nseg = (e1 > e0) ? ((e1 - 1) / epw - e0 / epw + 1) : 0;
     const float2* ml = a.ml + bh * a.jmax;
     const float* accp = a.acc + bh * a.jmax * kHeadDim + d;
@@ -654,43 +647,48 @@ cudaError_t decode_occupancy(bool dense, int G, int* ctas_per_sm) {
     return dense ? occupancy_of<true, 2>(ctas_per_sm) : occupancy_of<false, 2>(ctas_per_sm);
 }
 
-cudaError_t launch_bounds(const DecodeArgs& a, cudaStream_t stream) {
-    const dim3 grid((unsigned)((a.k_max + 255) / 256), (unsigned)((long)a.B * a.Hq));
-    bounds_kernel<<<grid, 256, 0, stream>>>(a);
-    return cudaGetLastError();
-}
-
 cudaError_t launch_union(const DecodeArgs& a, bool dense, cudaStream_t stream) {
     const size_t smem = union_smem(a);
     cudaError_t e;
     if (dense) {
         e = cudaFuncSetAttribute(union_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        union_kernel<true><<<a.nrt, kUnionThreads, smem, stream>>>(a);
+        e = launch_pdl(union_kernel<true>, dim3(a.nrt), dim3(kUnionThreads), smem, stream, a);
+        if (e != cudaSuccess) return e;
     } else {
         e = cudaFuncSetAttribute(union_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        union_kernel<false><<<a.nrt, kUnionThreads, smem, stream>>>(a);
+        e = launch_pdl(union_kernel<false>, dim3(a.nrt), dim3(kUnionThreads), smem, stream, a);
+        if (e != cudaSuccess) return e;
     }
     return cudaGetLastError();
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, bool dense, cudaStream_t stream) {
     const size_t smem = decode_smem();
-    const int ctas = a.total_warps;
-    if (a.G <= 8) {
-        if (dense) decode_kernel<true, 1><<<ctas, 32, smem, stream>>>(a);
-        else decode_kernel<false, 1><<<ctas, 32, smem, stream>>>(a);
-    } else {
-        if (dense) decode_kernel<true, 2><<<ctas, 32, smem, stream>>>(a);
-        else decode_kernel<false, 2><<<ctas, 32, smem, stream>>>(a);
-    }
-    return cudaGetLastError();
+    const dim3 grid(a.total_warps), block(32);
+    cudaError_t e;
+    if (a.G <= 8) e = dense ? launch_pdl(decode_kernel<true, 1>, grid, block, smem, stream, a)
+                            : launch_pdl(decode_kernel<false, 1>, grid, block, smem, stream, a);
+    else e = dense ? launch_pdl(decode_kernel<true, 2>, grid, block, smem, stream, a)
+                   : launch_pdl(decode_kernel<false, 2>, grid, block, smem, stream, a);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_merge(const DecodeArgs& a, cudaStream_t stream) {
-    merge_kernel<<<(unsigned)((long)a.B * a.Hq), kHeadDim, 0, stream>>>(a);
-    return cudaGetLastError();
+    cudaError_t e = launch_pdl(merge_kernel, dim3((unsigned)((long)a.B * a.Hq)), dim3(kHeadDim), 0, stream, a);
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+// Zeroes the per-group and global union-row totals that union_kernel accumulates.
+__global__ void __launch_bounds__(256) prep_kernel(DecodeArgs a) {
+    pdl_enter();
+    for (int i = threadIdx.x; i < 4 + a.B * a.Hkv; i += blockDim.x) a.hdr[i] = 0;
+}
+
+cudaError_t launch_prep(const DecodeArgs& a, cudaStream_t stream) {
+    cudaError_t e = launch_pdl(prep_kernel, dim3(1), dim3(256), 0, stream, a);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace sd

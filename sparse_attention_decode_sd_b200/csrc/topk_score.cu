@@ -80,6 +80,7 @@ __device__ __forceinline__ void load_k_row(const uint8_t* row, int c, int sw, ui
 template <int NT>
 __global__ void __launch_bounds__(kScoreThreads, 1) score_pass_kernel(TopkArgs a) {
     extern __shared__ __align__(1024) uint8_t smem[];
+    pdl_enter();
     const int page_bytes = kPageSize * a.Hkv * kRowBytes;
     const int stage_bytes = a.spp * page_bytes;
     const int S = a.stages;
@@ -223,11 +224,13 @@ cudaError_t launch_score_pass(const TopkArgs& a, int grid, cudaStream_t stream) 
     if (a.G <= 8) {
         cudaError_t e = cudaFuncSetAttribute(score_pass_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        score_pass_kernel<1><<<grid, kScoreThreads, smem, stream>>>(a);
+        e = launch_pdl(score_pass_kernel<1>, dim3(grid), dim3(kScoreThreads), smem, stream, a);
+        if (e != cudaSuccess) return e;
     } else {
         cudaError_t e = cudaFuncSetAttribute(score_pass_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        score_pass_kernel<2><<<grid, kScoreThreads, smem, stream>>>(a);
+        e = launch_pdl(score_pass_kernel<2>, dim3(grid), dim3(kScoreThreads), smem, stream, a);
+        if (e != cudaSuccess) return e;
     }
     return cudaGetLastError();
 }

@@ -153,6 +153,7 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(TopkArgs a) {
     int* scratch = hist + 4096;                  // [40]
     int* s_sel = scratch + 40;                   // [8]
     int* s_cnt = s_sel + 8;                      // [2][32] per-warp counts, double buffered
+    pdl_enter();
     uint32_t* lkey = reinterpret_cast<uint32_t*>(s_cnt + 64);
     int* lpos = reinterpret_cast<int*>(lkey + a.cap);
 
@@ -266,8 +267,8 @@ cudaError_t launch_select(const TopkArgs& a, cudaStream_t stream) {
     const size_t smem = select_smem(a);
     cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    select_kernel<<<a.B * a.Hq, kSelectThreads, smem, stream>>>(a);
-    return cudaGetLastError();
+    e = launch_pdl(select_kernel, dim3(a.B * a.Hq), dim3(kSelectThreads), smem, stream, a);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace sd
