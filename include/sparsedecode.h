@@ -100,11 +100,16 @@ SD_API sd_status sd_topk_index(const sd_shape* shape, const void* q, const void*
                         size_t workspace_bytes, int32_t* dev_status, void* stream);
 
 /* The two halves of sd_topk_index, for callers that schedule or time them separately.
- *   sd_topk_scores  writes s[b][h][i] (fp32) for every request that needs a selection
- *                   (1 <= k[b] < N_b) into the workspace; other rows are not written.
- *   sd_topk_select  reads those scores from the same workspace and writes idx exactly as
- *                   sd_topk_index does; it must follow sd_topk_scores on the same inputs and
- *                   workspace (stream order), with lens and k unchanged in between. */
+ *   sd_topk_scores  scores every position of every request that needs a selection
+ *                   (1 <= k[b] < N_b) and leaves in the workspace what the selection needs:
+ *                   the whole fp32 row s[b][h][0..N_b) when N_b <= 3 k_max + 4096, otherwise
+ *                   only the candidates (every score at or above a per-row threshold placed by a
+ *                   sample of the row) with their positions.  The workspace layout is internal.
+ *   sd_topk_select  reads those from the same workspace and writes idx exactly as sd_topk_index
+ *                   does (in the rare case a row's candidates cannot decide the selection, it
+ *                   recomputes that row from the q, K and page_table given to sd_topk_scores);
+ *                   it must follow sd_topk_scores on the same workspace (stream order), with
+ *                   q, K, page_table, lens and k unchanged in between. */
 SD_API sd_status sd_topk_scores(const sd_shape* shape, const void* q, const void* K, const int32_t* page_table,
                          const int32_t* lens, const int32_t* k, void* workspace, size_t workspace_bytes,
                          int32_t* dev_status, void* stream);
@@ -114,11 +119,12 @@ SD_API sd_status sd_topk_select(const sd_shape* shape, const int32_t* lens, cons
 /* sd_topk_index without a caller-provided workspace, for callers that cannot allocate device memory
  * (for example a plugin inside a host engine that passes it only inputs and outputs, or a service
  * whose device memory is fixed at start-up).  The pages have no counterpart of this entry point.
- *   Same inputs, outputs, checks and results as sd_topk_index.  The fp32 scores live in one
- *   file-scope device array of 32 MiB inside the library, held by every GPU that loads the library
+ *   Same inputs, outputs, checks and results as sd_topk_index.  The indexer's workspace lives in one
+ *   file-scope device array of 48 MiB inside the library, held by every GPU that loads the library
  *   until the process exits; the call allocates nothing.
- *   Limit: B * Hq * max_pages_per_req * 16 scores must fit in 32 MiB (8,388,608 floats), else
- *   SD_ERR_WORKSPACE and nothing is launched.
+ *   Limit: sd_workspace_size(shape, SD_OP_TOPK) must not exceed 48 MiB (for example one request of
+ *   64 query heads at 131072 positions and k_max 2621 fits), else SD_ERR_WORKSPACE and nothing is
+ *   launched.
  *   The first call on a device looks up the array's device address (cudaGetSymbolAddress) with that
  *   device current; make that first call before any stream capture.
  *   Every call on a device uses the same array, which keeps the last call's scores: calls whose
@@ -157,6 +163,11 @@ SD_API sd_status sd_append_kv(const sd_shape* shape, void* K, void* V, const int
 
 /* Static English text for a status code ("unknown status" for other values). */
 SD_API const char* sd_status_string(sd_status status);
+
+/* The CUDA runtime error (a cudaError_t value, with its name in *name if name is not NULL) behind
+ * the most recent SD_ERR_CUDA returned on the calling thread; 0 and "cudaSuccess" if there was none.
+ * The name is static text. */
+SD_API int32_t sd_last_cuda_error(const char** name);
 
 /* Library version, major * 10000 + minor * 100 + patch. */
 SD_API int32_t sd_version(void);

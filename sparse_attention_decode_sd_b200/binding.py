@@ -29,7 +29,7 @@ SD_OP_SPARSE = 2
 SD_OP_DENSE = 3
 
 EXPORTED = ("sd_workspace_size", "sd_topk_index", "sd_topk_scores", "sd_topk_select", "sd_topk_index_static",
-            "sd_sparse_decode", "sd_dense_decode", "sd_append_kv", "sd_status_string", "sd_version")
+            "sd_sparse_decode", "sd_dense_decode", "sd_append_kv", "sd_status_string", "sd_last_cuda_error", "sd_version")
 
 
 class SdShape(ctypes.Structure):
@@ -40,7 +40,11 @@ class SdShape(ctypes.Structure):
 
 class SdError(RuntimeError):
     def __init__(self, status: int, what: str):
-        super().__init__(f"{what}: {status_string(status)} (status {status})")
+        msg = f"{what}: {status_string(status)} (status {status})"
+        if status == SD_ERR_CUDA:
+            code, name = last_cuda_error()
+            msg += f": {name} ({code})"
+        super().__init__(msg)
         self.status = status
 
 
@@ -73,6 +77,8 @@ def load():
         f.restype = I32
     lib.sd_status_string.argtypes = [I32]
     lib.sd_status_string.restype = ctypes.c_char_p
+    lib.sd_last_cuda_error.argtypes = [ctypes.POINTER(ctypes.c_char_p)]
+    lib.sd_last_cuda_error.restype = I32
     lib.sd_version.argtypes = []
     lib.sd_version.restype = I32
     _lib = lib
@@ -81,6 +87,13 @@ def load():
 
 def status_string(status: int) -> str:
     return load().sd_status_string(int(status)).decode()
+
+
+def last_cuda_error() -> tuple[int, str]:
+    """(cudaError_t value, its name) behind the last SD_ERR_CUDA on this thread."""
+    name = ctypes.c_char_p()
+    code = load().sd_last_cuda_error(ctypes.byref(name))
+    return int(code), (name.value or b"").decode()
 
 
 def version() -> int:

@@ -15,6 +15,7 @@ namespace {
 constexpr int kMaxDevices = 64;
 constexpr size_t kSmemBudget = 227 * 1024;   // opt-in shared memory per CTA on sm_100
 constexpr int kSelectCapMax = 24 * 1024;      // select: candidate entries kept in shared memory
+constexpr size_t kScoreStageBytes = 65536;    // score pass: bytes per pipeline stage (whole pages)
 
 struct DeviceInfo {
     bool ready = false;
@@ -85,7 +86,26 @@ sd_status check_shape(const sd_shape* s, Dims* d) {
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-size_t topk_workspace(const Dims& d) { return align256((size_t)d.B * d.Hq * d.n_cap * sizeof(float)); }
+// indexer workspace, in order: candidate streams (B*Hq*n_cap fp32), per-(page, kv head) stream
+// offsets [B][Hkv][mstride] uint32, candidate masks [B][Hkv][mstride][G] uint16, thresholds
+// [B][Hq] fp32, input pointers [3]
+long topk_mstride(const Dims& d) { return ((long)d.max_pages + 7) & ~7L; }
+struct TopkLayout {
+    size_t cand, poff, pmask, tau, inputs, total;
+};
+TopkLayout topk_layout(const Dims& d) {
+    TopkLayout L;
+    const size_t rows = (size_t)d.B * d.Hq;
+    const size_t recs = (size_t)d.B * d.Hkv * topk_mstride(d);
+    L.cand = 0;
+    L.poff = align256(rows * d.n_cap * sizeof(float));
+    L.pmask = L.poff + align256(recs * sizeof(uint32_t));
+    L.tau = L.pmask + align256(recs * d.G * sizeof(uint16_t));
+    L.inputs = L.tau + align256(rows * sizeof(float));
+    L.total = L.inputs + align256(3 * sizeof(void*));
+    return L;
+}
+size_t topk_workspace(const Dims& d) { return topk_layout(d).total; }
 
 // decode workspace, in order: acc [B][Hq][jmax][128] fp32, ml [B][Hq][jmax] float2,
 // entries [nrt][kRange] uint2, counts [nrt], hdr [4] followed by per-group totals [B * Hkv]
@@ -107,7 +127,13 @@ size_t decode_workspace(const Dims& d) { return decode_layout(d).total; }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-sd_status launch_status(cudaError_t e) { return e == cudaSuccess ? SD_OK : SD_ERR_CUDA; }
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
+sd_status launch_status(cudaError_t e) {
+    if (e == cudaSuccess) return SD_OK;
+    g_last_cuda_error = e;
+    return SD_ERR_CUDA;
+}
 
 sd_status decode_common(const sd_shape* shape, const void* q, const void* K, const void* V, const int32_t* page_table,
                         const int32_t* lens, const int32_t* idx, float* out, void* workspace, size_t workspace_bytes,
@@ -207,7 +233,19 @@ sd_status topk_args(const sd_shape* shape, const void* q, const void* K, const i
     a->lens = lens;
     a->k = k;
     a->idx = idx;
-    a->scores = static_cast<float*>(workspace);
+    const TopkLayout L = topk_layout(d);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    if ((long)d.B * d.Hq * d.n_cap >= (1L << 32)) return SD_ERR_UNSUPPORTED;   // stream offsets are 32-bit
+    a->cand = reinterpret_cast<float*>(ws + L.cand);
+    a->poff = reinterpret_cast<uint32_t*>(ws + L.poff);
+    a->pmask = reinterpret_cast<uint16_t*>(ws + L.pmask);
+    a->tau = reinterpret_cast<float*>(ws + L.tau);
+    a->inputs = reinterpret_cast<const void**>(ws + L.inputs);
+    a->mstride = (int)topk_mstride(d);
+    // Rows with N_b <= 3 k_max + 4096 take every position as a candidate; longer rows keep the
+    // scores at or above a sampled threshold.
+    const long ccap = 3L * d.k_max + 4096;
+    a->ccap = (int)(ccap < d.n_cap ? ccap : d.n_cap);
     a->status = dev_status;
     a->B = d.B;
     a->Hq = d.Hq;
@@ -217,9 +255,10 @@ sd_status topk_args(const sd_shape* shape, const void* q, const void* K, const i
     a->num_pages = d.num_pages;
     a->k_max = d.k_max;
     a->n_cap = d.n_cap;
-    // score pass: pipeline stages of >= 32 KB, as deep as the shared memory allows (<= 6)
+    // score pass: pipeline stages of whole pages, about kScoreStageBytes each, as many as the shared
+    // memory holds (2 to 6)
     const size_t page_bytes = (size_t)kPageSize * d.Hkv * kRowBytes;
-    a->spp = (int)(page_bytes >= 32768 ? 1 : 32768 / page_bytes);
+    a->spp = (int)(page_bytes >= kScoreStageBytes ? 1 : kScoreStageBytes / page_bytes);
     const size_t fixed = sizeof(int) * (d.B + 1 + 40) + 1024;
     const size_t stage_bytes = page_bytes * a->spp;
     a->stages = (int)((kSmemBudget - fixed) / (stage_bytes + 2 * sizeof(uint64_t)));
@@ -242,7 +281,10 @@ sd_status sd_topk_scores(const sd_shape* shape, const void* q, const void* K, co
     sd_status st = topk_args(shape, q, K, page_table, lens, k, nullptr, workspace, workspace_bytes, dev_status, true,
                              false, &a, &di);
     if (st != SD_OK) return st;
-    return launch_status(launch_score_pass(a, di.sms, static_cast<cudaStream_t>(stream)));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    st = launch_status(launch_threshold(a, s));
+    if (st != SD_OK) return st;
+    return launch_status(launch_score_pass(a, di.sms, s));
 }
 
 sd_status sd_topk_select(const sd_shape* shape, const int32_t* lens, const int32_t* k, int32_t* idx, void* workspace,
@@ -264,6 +306,8 @@ sd_status sd_topk_index(const sd_shape* shape, const void* q, const void* K, con
                              &a, &di);
     if (st != SD_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    st = launch_status(launch_threshold(a, s));
+    if (st != SD_OK) return st;
     st = launch_status(launch_score_pass(a, di.sms, s));
     if (st != SD_OK) return st;
     return launch_status(launch_select(a, s));
@@ -322,6 +366,11 @@ const char* sd_status_string(sd_status status) {
         case SD_ERR_ORDER: return "index row not strictly ascending";
         default: return "unknown status";
     }
+}
+
+int32_t sd_last_cuda_error(const char** name) {
+    if (name != nullptr) *name = cudaGetErrorName(g_last_cuda_error);
+    return (int32_t)g_last_cuda_error;
 }
 
 int32_t sd_version(void) { return 100; }

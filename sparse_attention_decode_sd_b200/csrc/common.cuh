@@ -94,6 +94,39 @@ __device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32
         : "memory");
 }
 
+// Tiled 4-D tensor copy global -> shared (TMA), completing its bytes on `bar`.  The innermost
+// coordinate x times the element size must be a multiple of 16 bytes; dst is 128-byte aligned
+// (1024-byte aligned for a 128-byte swizzled map).
+__device__ __forceinline__ void tma_load_4d(void* dst, const void* tmap, int x, int y, int z, int w, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], "
+        "[%6];\n" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_addr(bar))
+        : "memory");
+}
+
+// ---------------------------------------------------------------------------------------------
+// Thread-block clusters: rank, cluster-wide barrier, distributed shared memory stores.
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;\n" : "=r"(r));
+    return r;
+}
+// All threads of all CTAs of the cluster; writes before it are visible to every CTA after it.
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;\n" ::: "memory");
+}
+// Shared-memory address `saddr` of this CTA mapped to the same variable in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_shared_rank(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void st_cluster_u16(uint32_t addr, uint16_t v) {
+    asm volatile("st.shared::cluster.u16 [%0], %1;\n" ::"r"(addr), "h"(v) : "memory");
+}
+
 // ---------------------------------------------------------------------------------------------
 // Tensor-core fragments (mma.sync m16n8k16, bf16 in, fp32 accumulate) and ldmatrix.
 // ---------------------------------------------------------------------------------------------
@@ -132,6 +165,11 @@ __device__ __forceinline__ uint32_t float_key(float x) {
     uint32_t u = __float_as_uint(x);
     if (u == 0x80000000u) u = 0u;
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Inverse of float_key.
+__device__ __forceinline__ float key_float(uint32_t key) {
+    return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
 }
 
 // ---------------------------------------------------------------------------------------------

@@ -8,6 +8,9 @@
 
 namespace sd {
 
+constexpr int kSample = 2048;         // sampled positions per row for the candidate threshold
+constexpr int kThresholdCluster = 8;  // CTAs (one cluster) that score one group's sample
+
 struct TopkArgs {
     const __nv_bfloat16* q;
     const __nv_bfloat16* K;
@@ -15,16 +18,28 @@ struct TopkArgs {
     const int32_t* lens;
     const int32_t* k;
     int32_t* idx;
-    float* scores;      // workspace: fp32 [B][Hq][n_cap]
+    float* cand;        // workspace, B*Hq*n_cap floats: candidate scores, one sequential stream per
+                        // score-pass warp; the candidates of unit (page p, kv head) are stored
+                        // head-major from cand[poff[...p]], each head's in position order
+    uint32_t* poff;     // workspace [B][Hkv][mstride]: where each (page, kv head) unit's candidates start
+    uint16_t* pmask;    // workspace [B][Hkv][mstride][G]: bit i = position p*16 + i of that head is a candidate
+    float* tau;         // workspace [B][Hq]: candidate threshold (scores >= tau are candidates;
+                        // -inf: every position)
+    const void** inputs;   // workspace [3]: q, K and page_table of the last score pass (the select
+                           // step reads them from here when it has to recompute a row)
     int32_t* status;
     int B, Hq, Hkv, G, max_pages, num_pages, k_max;
     long n_cap;         // max_pages * page size: row stride of the score buffer
+    int mstride;        // pages per (request, kv head) record row (max_pages rounded up to 8)
+    int ccap;           // rows with N_b <= ccap take every position as a candidate
     int spp;            // pages per pipeline stage of the score pass
     int stages;         // pipeline depth of the score pass
     int cap;            // select: candidate entries that fit in shared memory
 };
 
 size_t score_pass_smem(const TopkArgs& a);
+size_t threshold_smem(const TopkArgs& a);
+cudaError_t launch_threshold(const TopkArgs& a, cudaStream_t stream);
 size_t select_smem(const TopkArgs& a);
 cudaError_t launch_score_pass(const TopkArgs& a, int grid, cudaStream_t stream);
 cudaError_t launch_select(const TopkArgs& a, cudaStream_t stream);

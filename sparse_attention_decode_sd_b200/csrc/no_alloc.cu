@@ -4,9 +4,10 @@
 // planned once at start-up and may not grow; code that runs on the calling thread while that thread
 // must not call cudaMalloc (which synchronises the device and is not a stream operation).
 //
-// The fp32 score rows live instead in one file-scope device array of kStaticScoreBytes (32 MiB).
-// Every GPU that loads this library holds that array until the process exits.  The call itself
-// allocates nothing: no cudaMalloc, no cudaFree, no allocating library routine.
+// The indexer's workspace (fp32 score rows or candidate pairs, thresholds, candidate counts) lives instead in one
+// file-scope device array of kStaticScratchBytes (48 MiB).  Every GPU that loads this library holds
+// that array until the process exits.  The call itself allocates nothing: no cudaMalloc, no
+// cudaFree, no allocating library routine.
 #include <mutex>
 
 #include "common.cuh"
@@ -14,12 +15,12 @@
 
 namespace {
 
-constexpr size_t kStaticScoreBytes = 32u << 20;   // 32 MiB = 8,388,608 fp32 scores
+constexpr size_t kStaticScratchBytes = 48u << 20;   // 48 MiB
 constexpr int kMaxDevices = 64;
 
 // The scratch.  In host code this name is only a host-side handle for the symbol, not a device
 // address: the device address comes from cudaGetSymbolAddress below.
-static __device__ __align__(256) float sd_static_scores[kStaticScoreBytes / sizeof(float)];
+static __device__ __align__(256) float sd_static_scratch[kStaticScratchBytes / sizeof(float)];
 
 std::mutex g_static_mu;
 void* g_static_ptr[kMaxDevices] = {};
@@ -33,7 +34,7 @@ sd_status static_scratch(void** out) {
     std::lock_guard<std::mutex> lock(g_static_mu);
     if (g_static_ptr[dev] == nullptr) {
         void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, sd_static_scores) != cudaSuccess || p == nullptr) return SD_ERR_CUDA;
+        if (cudaGetSymbolAddress(&p, sd_static_scratch) != cudaSuccess || p == nullptr) return SD_ERR_CUDA;
         g_static_ptr[dev] = p;
     }
     *out = g_static_ptr[dev];
@@ -48,11 +49,11 @@ extern "C" sd_status sd_topk_index_static(const sd_shape* shape, const void* q, 
     size_t need = 0;
     sd_status st = sd_workspace_size(shape, SD_OP_TOPK, &need);
     if (st != SD_OK) return st;
-    if (need > kStaticScoreBytes) return SD_ERR_WORKSPACE;   // B * Hq * max_pages * 16 scores exceed 32 MiB
+    if (need > kStaticScratchBytes) return SD_ERR_WORKSPACE;   // the shape's indexer workspace exceeds 48 MiB
     void* scratch = nullptr;
     st = static_scratch(&scratch);
     if (st != SD_OK) return st;
-    // Nothing in the scratch has to start at zero: the score pass writes every score the
-    // selection reads.  Successive calls reuse the same array.
-    return sd_topk_index(shape, q, K, page_table, lens, k, idx, scratch, kStaticScoreBytes, dev_status, stream);
+    // Nothing in the scratch has to start at zero: each call resets the counters it accumulates and
+    // writes every score and candidate its selection reads.  Successive calls reuse the same array.
+    return sd_topk_index(shape, q, K, page_table, lens, k, idx, scratch, kStaticScratchBytes, dev_status, stream);
 }

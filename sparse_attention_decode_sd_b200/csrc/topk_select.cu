@@ -2,11 +2,13 @@
 // summary sec. 2): per (request, query head), the k highest scores of the row the score pass wrote,
 // ties at the k-th score going to the lower position, emitted as ascending positions.
 //
-// select_kernel, one CTA per (b, h): a strided sample of the scores places a candidate threshold;
-// one pass over the row compacts every key at or above it, in position order, into shared memory;
-// an exact radix select over order-preserving 32-bit keys (12 + 12 + 8 bits) finds the k-th key
-// there, and an ordered compaction writes the ascending positions.  If the sample misplaced the
-// threshold, the exact select runs over the whole row in global memory instead.
+// select_kernel, one CTA per (b, h), reads the row's candidates as the score pass left them (a
+// 16-bit mask per page and head, scores in the score-pass warps' streams).  If the threshold
+// admitted fewer than k candidates (rare), it selects from scores recomputed on the fly.  Usual case: the
+// candidates are compacted in position order into shared memory, where an exact radix select over
+// order-preserving 32-bit keys (12 + 12 + 8 bits) finds the k-th key and an ordered compaction
+// writes the ascending positions.  If they do not fit, the same select runs on the masked row in
+// global memory (L2), with block scans putting the output in order.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -18,13 +20,6 @@ constexpr int kSelectItems = 4;   // consecutive elements per thread per tile of
 // ---------------------------------------------------------------------------------------------
 // select
 // ---------------------------------------------------------------------------------------------
-struct GlobalKeys {   // the fp32 scores of one (b, h), read from the workspace
-    const float* sc;
-    int n;
-    __device__ __forceinline__ int size() const { return n; }
-    __device__ __forceinline__ uint32_t key(int j) const { return float_key(sc[j]); }
-    __device__ __forceinline__ int pos(int j) const { return j; }
-};
 struct SharedKeys {   // (key, position) list in shared memory, ascending positions
     const uint32_t* k;
     const int* p;
@@ -64,36 +59,72 @@ __device__ __forceinline__ void select_bin(const int* hist, int nbins, int targe
     __syncthreads();
 }
 
-// Exact radix select: the key T of the target-th largest element of src (12 + 12 + 8 bit digits)
-// and the number of elements with a key greater than T.
-template <class Src>
-__device__ void radix_find(const Src& src, int target, int* hist, int* scratch, int* s_sel, uint32_t* T_out,
-                           int* greater_out) {
-    const int tid = threadIdx.x, nthr = blockDim.x;
-    const int n = src.size();
-    uint32_t prefix = 0;
-    int greater = 0;
-    // digits: key bits 31..20, then 19..8, then 7..0
-    const int shifts[3] = {20, 8, 0};
-    const int widths[3] = {12, 12, 8};
+// Exact radix select over the keys a thread visits with visit(f) (f(key) per element): the key T
+// of the target-th largest element (1 <= target <= count) and the number of elements with a key
+// greater than T.  The keys' range is found first and the digits (up to 12 bits each) start at the
+// highest bit in which the smallest and largest key differ: candidates cluster just above a
+// threshold, so a fixed top digit would pile them into a few contended histogram bins.
+template <class Visit>
+__device__ void radix_select(Visit visit, int target, int* hist, int* scratch, int* s_sel, uint32_t* T_out,
+                             int* greater_out) {
+    const int tid = threadIdx.x, nthr = blockDim.x, lane = tid & 31;
+    uint32_t kmin = 0xffffffffu, kmax = 0u;
+    visit([&](uint32_t key) {
+        kmin = min(kmin, key);
+        kmax = max(kmax, key);
+    });
 #pragma unroll
-    for (int d = 0; d < 3; ++d) {
-        const int nb = 1 << widths[d];
+    for (int o = 16; o > 0; o >>= 1) {
+        kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
+        kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+    }
+    unsigned int* range = reinterpret_cast<unsigned int*>(s_sel + 2);
+    if (tid == 0) {
+        range[0] = 0xffffffffu;
+        range[1] = 0u;
+    }
+    __syncthreads();
+    if (lane == 0) {
+        atomicMin(&range[0], kmin);
+        atomicMax(&range[1], kmax);
+    }
+    __syncthreads();
+    kmin = range[0];
+    kmax = range[1];
+    __syncthreads();
+    const uint32_t diff = kmin ^ kmax;
+    int top = diff ? 31 - __clz(diff) : -1;   // highest bit that differs; above it every key is kmin's
+    uint32_t prefix = top >= 31 ? 0u : (kmin >> (top + 1)) << (top + 1);
+    int greater = 0;
+    while (top >= 0) {
+        const int w = min(12, top + 1), sh = top + 1 - w;
+        const int nb = 1 << w;
         for (int i = tid; i < nb; i += nthr) hist[i] = 0;
         __syncthreads();
-        const int hs = shifts[d] + widths[d];   // bits above this digit must equal the prefix
-        for (int j = tid; j < n; j += nthr) {
-            const uint32_t key = src.key(j);
-            if (hs >= 32 || (key >> hs) == prefix) atomicAdd(&hist[(key >> shifts[d]) & (uint32_t)(nb - 1)], 1);
-        }
+        visit([&](uint32_t key) {
+            if (top >= 31 || (key >> (top + 1)) == (prefix >> (top + 1)))
+                atomicAdd(&hist[(key >> sh) & (uint32_t)(nb - 1)], 1);
+        });
         __syncthreads();
         select_bin(hist, nb, target - greater, scratch, s_sel);
-        prefix = (prefix << widths[d]) | (uint32_t)s_sel[0];
+        prefix |= (uint32_t)s_sel[0] << sh;
         greater += s_sel[1];
+        top = sh - 1;
         __syncthreads();
     }
-    *T_out = prefix;
+    *T_out = prefix;       // all keys equal: T is that key, none greater
     *greater_out = greater;
+}
+
+template <class Src>
+__device__ __forceinline__ void radix_find(const Src& src, int target, int* hist, int* scratch, int* s_sel,
+                                           uint32_t* T_out, int* greater_out) {
+    const int n = src.size();
+    radix_select(
+        [&](auto f) {
+            for (int j = threadIdx.x; j < n; j += blockDim.x) f(src.key(j));
+        },
+        target, hist, scratch, s_sel, T_out, greater_out);
 }
 
 // Writes the selected positions of src in ascending order to row[0..take): keys above T, plus the
@@ -145,19 +176,158 @@ __device__ void select_exact(const Src& src, int take, int32_t* row, int* hist, 
     emit_selected(src, T, take - greater, take, row, scratch);
 }
 
-constexpr int kSample = 2048;   // strided sample of the scores used to place the candidate threshold
+// The candidates of row (b, h) as the score pass left them.  Per page p of the row's KV head:
+// pmask[p][col] marks which of the page's 16 positions are candidates for head col = h mod G, and
+// the page's candidates of all G heads sit head by head from cand[poff[p]] on.  Thread t of the
+// block owns the pages [t*per, (t+1)*per) and visits its candidates in ascending position order,
+// so a block scan over per-thread counts orders the whole row.
+struct StreamRow {
+    const float* cand;
+    const uint32_t* poff;
+    const uint16_t* pmask;
+    int G, col;
+    uint32_t limit;   // floats in the stream buffer: a record pointing past it is skipped (it can only
+                      // come from a score pass that stopped early, which reported that)
+    int p0, p1;       // this thread's pages
+    __device__ StreamRow(const TopkArgs& a, long bh, int n) {
+        const int b = (int)(bh / a.Hq), h = (int)(bh % a.Hq), kvh = h / a.G;
+        const long rec = ((long)b * a.Hkv + kvh) * a.mstride;
+        cand = a.cand;
+        poff = a.poff + rec;
+        pmask = a.pmask + rec * a.G;
+        G = a.G;
+        col = h - kvh * a.G;
+        limit = (uint32_t)((long)a.B * a.Hq * a.n_cap);
+        const int np = (n + kPageSize - 1) / kPageSize;
+        const int per = (np + (int)blockDim.x - 1) / (int)blockDim.x;
+        p0 = min(np, (int)threadIdx.x * per);
+        p1 = min(np, p0 + per);
+    }
+    __device__ __forceinline__ uint32_t mask(int p) const { return pmask[(long)p * G + col]; }
+    __device__ __forceinline__ int count() const {
+        int c = 0;
+        for (int p = p0; p < p1; ++p) c += __popc(mask(p));
+        return c;
+    }
+    template <class F>
+    __device__ __forceinline__ void for_each(F f) const {
+        for (int p = p0; p < p1; ++p) {
+            uint32_t m = mask(p);
+            if (m == 0u) continue;
+            uint32_t base = poff[p];
+            if ((G & 7) == 0) {   // records of 16-byte multiples: masks of the heads before col by vector
+                const uint4* r = reinterpret_cast<const uint4*>(pmask + (long)p * G);
+                for (int q = 0; q * 8 < col; ++q) {
+                    const uint4 v = r[q];
+                    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+                    const int below = min(8, col - q * 8);   // masks of this vector before col
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        const int nbits = min(32, max(0, 16 * (below - 2 * t)));
+                        base += __popc(nbits >= 32 ? w[t] : (w[t] & ((1u << nbits) - 1u)));
+                    }
+                }
+            } else {
+                for (int hh = 0; hh < col; ++hh) base += __popc((uint32_t)pmask[(long)p * G + hh]);
+            }
+            if ((unsigned long)base + __popc(m) > limit) continue;
+            const float* sp = cand + base;
+            for (int i = 0; m; ++i) {
+                const int bit = __ffs(m) - 1;
+                m &= m - 1u;
+                f(float_key(sp[i]), p * kPageSize + bit);
+            }
+        }
+    }
+};
+
+// Rare fallback, when the threshold admitted fewer candidates than k: every score of row (b, h)
+// recomputed on the fly from q and K in each pass (a fixed order of fp32 operations, so every pass
+// sees the same values).  Thread t owns the positions [t*per, (t+1)*per).  q (fp32, in shared memory
+// at qs) and the inputs are the ones the score pass recorded in the workspace.
+struct RecomputedRow {
+    const __nv_bfloat16* K;
+    const int32_t* ptrow;
+    const float* qs;
+    int Hkv, kvh, num_pages;
+    int i0, i1;
+    __device__ RecomputedRow(const TopkArgs& a, long bh, int n, const float* q_smem) {
+        const int b = (int)(bh / a.Hq), h = (int)(bh % a.Hq);
+        K = static_cast<const __nv_bfloat16*>(a.inputs[1]);
+        ptrow = static_cast<const int32_t*>(a.inputs[2]) + (long)b * a.max_pages;
+        qs = q_smem;
+        Hkv = a.Hkv;
+        kvh = h / a.G;
+        num_pages = a.num_pages;
+        const int per = (n + (int)blockDim.x - 1) / (int)blockDim.x;
+        i0 = min(n, (int)threadIdx.x * per);
+        i1 = min(n, i0 + per);
+    }
+    template <class F>
+    __device__ __forceinline__ void for_each(F f) const {
+        for (int i = i0; i < i1; ++i) {
+            int page = __ldg(ptrow + i / kPageSize);
+            if (page < 0 || page >= num_pages) page = 0;   // reported by the score pass
+            const uint4* row =
+                reinterpret_cast<const uint4*>(K + (((long)page * kPageSize + (i % kPageSize)) * Hkv + kvh) * kHeadDim);
+            float d = 0.f;
+#pragma unroll 4
+            for (int ch = 0; ch < kHeadDim / 8; ++ch) {
+                const uint4 v = __ldg(row + ch);
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int t = 0; t < 4; ++t)
+                    d = fmaf(bf16_hi(w[t]), qs[ch * 8 + 2 * t + 1], fmaf(bf16_lo(w[t]), qs[ch * 8 + 2 * t], d));
+            }
+            f(float_key(d), i);
+        }
+    }
+};
+
+// Selection straight from a source visited with for_each in thread-ordered position order (any
+// number of candidates): radix select, then the ascending positions through two block scans (ties
+// first, then the selected).
+template <class Src>
+__device__ void select_masked(const Src& src, int take, int32_t* row, int* hist, int* scratch, int* s_sel) {
+    uint32_t T;
+    int greater;
+    radix_select([&](auto f) { src.for_each([&](uint32_t key, int) { f(key); }); }, take, hist, scratch, s_sel, &T,
+                 &greater);
+    const int quota = take - greater;
+    int tc = 0;
+    src.for_each([&](uint32_t key, int) { tc += key == T; });
+    int ttot;
+    const int tie_before = block_exclusive_scan(tc, scratch, &ttot);
+    int sc = 0;
+    {
+        int tb = tie_before;
+        src.for_each([&](uint32_t key, int) {
+            if (key > T) ++sc;
+            else if (key == T) sc += (tb++ < quota);
+        });
+    }
+    int stot;
+    int out = block_exclusive_scan(sc, scratch, &stot);
+    int tb = tie_before;
+    src.for_each([&](uint32_t key, int pos) {
+        const bool keep = key > T || (key == T && tb++ < quota);
+        if (keep) {
+            if (out < take) row[out] = pos;
+            ++out;
+        }
+    });
+}
 
 __global__ void __launch_bounds__(kSelectThreads) select_kernel(TopkArgs a) {
     extern __shared__ __align__(1024) uint8_t smem[];
     int* hist = reinterpret_cast<int*>(smem);   // [4096]
     int* scratch = hist + 4096;                  // [40]
     int* s_sel = scratch + 40;                   // [8]
-    int* s_cnt = s_sel + 8;                      // [2][32] per-warp counts, double buffered
+    uint32_t* lkey = reinterpret_cast<uint32_t*>(s_sel + 8);   // [cap]
+    int* lpos = reinterpret_cast<int*>(lkey + a.cap);           // [cap]
     pdl_enter();
-    uint32_t* lkey = reinterpret_cast<uint32_t*>(s_cnt + 64);
-    int* lpos = reinterpret_cast<int*>(lkey + a.cap);
 
-    const int tid = threadIdx.x, nthr = blockDim.x, lane = tid & 31, warp = tid >> 5, nwarps = nthr >> 5;
+    const int tid = threadIdx.x, nthr = blockDim.x;
     const long bh = blockIdx.x;
     const int b = (int)(bh / a.Hq);
     int32_t* row = a.idx + bh * a.k_max;
@@ -173,87 +343,28 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(TopkArgs a) {
         for (int i = tid; i < a.k_max; i += nthr) row[i] = (i < n) ? i : -1;
         return;
     }
-    const float* sc = a.scores + bh * a.n_cap;
-
-    // Candidate threshold tau: the j-th largest key of a strided sample, j chosen so that the keys
-    // >= tau are expected to number about 1.25 take + 16 sample strides (many standard deviations
-    // above take, well below the shared-memory capacity).  Small rows take every key.
-    uint32_t tau = 0u;
-    if (n > a.cap) {
-        const int stride = n / kSample;
-        uint32_t* skey = lkey;   // the sample lives in the candidate buffer until the pass below
-        for (int i = tid; i < kSample; i += nthr) skey[i] = float_key(sc[(long)i * stride]);
+    StreamRow src(a, bh, n);
+    const int cnt = src.count();
+    int total;
+    int off = block_exclusive_scan(cnt, scratch, &total);
+    if (total < take) {
+        // the threshold admitted fewer candidates than k: select from scores recomputed on the fly
+        float* qs = reinterpret_cast<float*>(lkey);
+        const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.inputs[0]) + bh * kHeadDim;
+        for (int i = tid; i < kHeadDim; i += nthr) qs[i] = __bfloat162float(q[i]);
         __syncthreads();
-        const long want = ((long)take * kSample + n - 1) / n;
-        const int j = (int)min((long)kSample, want + want / 4 + 16);
-        int greater;
-        radix_find(SharedKeys{skey, nullptr, kSample}, j, hist, scratch, s_sel, &tau, &greater);
-    }
-
-    // One pass: ordered compaction of every key >= tau into shared memory.  A tile is nthr * 16
-    // consecutive keys; thread t owns 16 consecutive keys of it (four 16-byte loads in flight).
-    constexpr int kPerThread = 16;
-    int base = 0;
-    int buf = 0;
-    for (int i0 = 0; i0 < n; i0 += nthr * kPerThread) {
-        const int i = i0 + tid * kPerThread;
-        uint32_t key[kPerThread];
-        if (i + kPerThread <= n) {
-            float4 v[kPerThread / 4];
-#pragma unroll
-            for (int u = 0; u < kPerThread / 4; ++u) v[u] = *reinterpret_cast<const float4*>(sc + i + 4 * u);
-#pragma unroll
-            for (int u = 0; u < kPerThread / 4; ++u) {
-                key[4 * u + 0] = float_key(v[u].x);
-                key[4 * u + 1] = float_key(v[u].y);
-                key[4 * u + 2] = float_key(v[u].z);
-                key[4 * u + 3] = float_key(v[u].w);
-            }
-        } else {
-#pragma unroll
-            for (int e = 0; e < kPerThread; ++e) key[e] = (i + e < n) ? float_key(sc[i + e]) : 0u;
-        }
-        int cnt = 0;
-#pragma unroll
-        for (int e = 0; e < kPerThread; ++e) cnt += (i + e < n) && key[e] >= tau;
-        int incl = cnt;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int t = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += t;
-        }
-        if (lane == 31) s_cnt[buf * 32 + warp] = incl;
+        select_masked(RecomputedRow(a, bh, n, qs), take, row, hist, scratch, s_sel);
+    } else if (total <= a.cap) {
+        // the usual case: the candidates, in position order, into shared memory
+        src.for_each([&](uint32_t key, int pos) {
+            lkey[off] = key;
+            lpos[off] = pos;
+            ++off;
+        });
         __syncthreads();
-        const int wc = (lane < nwarps) ? s_cnt[buf * 32 + lane] : 0;
-        int wincl = wc;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int t = __shfl_up_sync(0xffffffffu, wincl, o);
-            if (lane >= o) wincl += t;
-        }
-        const int wbase = __shfl_sync(0xffffffffu, wincl - wc, warp);
-        const int tile_tot = __shfl_sync(0xffffffffu, wincl, 31);
-        if (cnt > 0) {
-            int w = base + wbase + incl - cnt;
-#pragma unroll
-            for (int e = 0; e < kPerThread; ++e)
-                if ((i + e < n) && key[e] >= tau) {
-                    if (w < a.cap) {
-                        lkey[w] = key[e];
-                        lpos[w] = i + e;
-                    }
-                    ++w;
-                }
-        }
-        base += tile_tot;
-        buf ^= 1;
-    }
-    __syncthreads();
-    if (base >= take && base <= a.cap) {
-        select_exact(SharedKeys{lkey, lpos, base}, take, row, hist, scratch, s_sel);
+        select_exact(SharedKeys{lkey, lpos, total}, take, row, hist, scratch, s_sel);
     } else {
-        // the sample misplaced tau (too few or too many candidates): exact select on the full row
-        select_exact(GlobalKeys{sc, n}, take, row, hist, scratch, s_sel);
+        select_masked(src, take, row, hist, scratch, s_sel);
     }
     for (int i = take + tid; i < a.k_max; i += nthr) row[i] = -1;
 }
@@ -261,7 +372,7 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(TopkArgs a) {
 // ---------------------------------------------------------------------------------------------
 // host launcher
 // ---------------------------------------------------------------------------------------------
-size_t select_smem(const TopkArgs& a) { return sizeof(int) * (4096 + 40 + 8 + 64) + (size_t)a.cap * 8; }
+size_t select_smem(const TopkArgs& a) { return sizeof(int) * (4096 + 40 + 8) + (size_t)a.cap * 8; }
 
 cudaError_t launch_select(const TopkArgs& a, cudaStream_t stream) {
     const size_t smem = select_smem(a);

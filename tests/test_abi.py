@@ -55,6 +55,10 @@ def test_status_strings_and_version(lib):
     assert sdb.version() >= 100
 
 
+def test_last_cuda_error_starts_clear(lib):
+    assert sdb.last_cuda_error() == (0, "cudaSuccess")
+
+
 def _shape(**kw):
     base = dict(B=4, Hq=64, Hkv=8, max_pages=8192, k_max=2621, num_pages=32768)
     base.update(kw)
@@ -65,7 +69,11 @@ def _shape(**kw):
 def test_workspace_sizes(lib):
     s = _shape()
     topk = sdb.sd_workspace_size(s, sdb.SD_OP_TOPK)
-    assert topk == 4 * 64 * 8192 * 16 * 4                  # fp32 scores [B][Hq][n_cap]
+    rows = 4 * 64
+    scores = rows * 8192 * 16 * 4                          # fp32 candidate streams, B*Hq*n_cap
+    recs = 4 * 8 * 8192                                    # (request, kv head, page) records
+    small = recs * 4 + recs * 8 * 2 + rows * 4 + 3 * 8     # stream offsets, masks per head, thresholds, pointers
+    assert scores + small <= topk <= scores + small + 5 * 256
     sparse = sdb.sd_workspace_size(s, sdb.SD_OP_SPARSE)
     assert sparse == sdb.sd_workspace_size(s, sdb.SD_OP_DENSE)
     slots = 4 * 64 * (8192 * 16 // 128 + 1)

@@ -87,7 +87,8 @@ def test_decode_arbitrary_index_sets():
 @pytest.mark.parametrize("n,k", [(3000, 100), (40000, 100), (40000, 39999)])
 def test_exact_ties_go_to_lower_positions(n, k):
     """Identical K rows: every score ties, so the selection is exactly positions 0..k-1.  With N
-    large the tied bin overflows the shared-memory candidate list (streaming refinement path)."""
+    large every position passes the candidate threshold, the score pass's candidate segments
+    overflow, and the row is recomputed and selected in full."""
     w_cpu = wl.make_workload(1, 4, 1, n, k, seed=7)
     w_cpu.K[:] = w_cpu.K[0, 0, 0]
     w = w_cpu.to(DEV)
@@ -96,6 +97,40 @@ def test_exact_ties_go_to_lower_positions(n, k):
     assert r.device_status() == 0
     assert (idx[0, :, :k] == np.arange(k)).all()
     assert (idx[0, :, k:] == -1).all()
+
+
+def test_partial_ties_resolved_among_candidates():
+    """K rows drawn from 50 distinct vectors: each score value is shared by about 800 positions, so
+    the k-th score ties many times over while the candidates still fit their segments.  The
+    selection is unique (lowest positions among the tied) and must equal the oracle's exactly."""
+    n, k = 40000, 100
+    w_cpu = wl.make_workload(2, 8, 2, [n, n - 4321], k, seed=14, page_order="shuffled")
+    g = torch.Generator().manual_seed(15)
+    for b in range(2):
+        nb = int(w_cpu.lens[b])
+        pos = torch.arange(nb)
+        pages = w_cpu.page_table[b].long()[pos // w_cpu.P]
+        slots = pos % w_cpu.P
+        src = torch.randint(0, 50, (nb,), generator=g)
+        K0 = w_cpu.K[pages[:50], slots[:50]].clone()   # [50][Hkv][128]
+        w_cpu.K[pages, slots] = K0[src]
+    w = w_cpu.to(DEV)
+    r = gh.Runner(w)
+    idx = r.topk().cpu().numpy()
+    assert r.device_status() == 0
+    ref = oracle.topk(w_cpu.shape(), w_cpu.q, w_cpu.K, w_cpu.page_table, w_cpu.lens, w_cpu.k)
+    assert np.array_equal(idx, ref)
+
+
+def test_many_requests_per_score_cta():
+    """512 requests alternating between thresholded rows (N = 4200 > 3 k + 4096) and rows whose every
+    position is a candidate (N = 1000): each score-pass CTA spans four or five requests, so every
+    consumer warp's candidate stream crosses request boundaries."""
+    B = 512
+    lens = [4200 if b % 2 == 0 else 1000 for b in range(B)]
+    lens[5] = 4199
+    w_cpu = wl.make_workload(B, 2, 1, lens, 3, seed=16, page_order="shuffled")
+    _run_small(w_cpu, check_dense=False)
 
 
 def test_sampled_threshold_misplaced_falls_back():

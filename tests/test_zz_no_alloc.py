@@ -1,6 +1,7 @@
 """sd_topk_index_static: the top-k indexer for callers that cannot allocate device memory (a plugin
-handed only its inputs and outputs, a service with a fixed device-memory plan).  It keeps its fp32
-scores in a 32 MiB array inside the library instead of a caller workspace.
+handed only its inputs and outputs, a service with a fixed device-memory plan).  It keeps its
+workspace (score rows, candidate counts) in a 48 MiB array inside the library instead of a caller
+workspace.
 
 Checked through the C ABI against sd_topk_index with an ordinary workspace, on two calls in a row
 with different shapes (the second call reuses the array the first one filled), and the size limit
@@ -40,14 +41,14 @@ def _both(w):
 
 def test_static_scratch_matches_workspace_version_twice():
     first = wl.make_workload(2, 16, 4, [9000, 5000], [180, 100], seed=41, device="cuda")
-    second = wl.make_workload(1, 64, 8, 131072, 2621, seed=42, structure="sinks3", device="cuda")   # fills 32 MiB
+    second = wl.make_workload(1, 64, 8, 131072, 2621, seed=42, structure="sinks3", device="cuda")   # just over 32 MiB
     for w in (first, second):
         ref, got = _both(w)
         assert torch.equal(ref, got)   # integer output: identical
 
 
 def test_static_scratch_rejects_shapes_beyond_its_size():
-    shape = sdb.make_shape(2, 64, 8, 8192, 2621, 16384)   # 2 * 64 * 131072 scores = 64 MiB
+    shape = sdb.make_shape(2, 64, 8, 8192, 2621, 16384)   # 2 * 64 * 131072 scores alone = 64 MiB
     fake = ctypes.c_void_p(1 << 20)
     status = sdb.load().sd_topk_index_static(ctypes.byref(shape), fake, fake, fake, fake, fake, fake, fake, None)
     assert status == sdb.SD_ERR_WORKSPACE
