@@ -86,21 +86,18 @@ sd_status check_shape(const sd_shape* s, Dims* d) {
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-// indexer workspace, in order: candidate streams (B*Hq*n_cap fp32), per-(page, kv head) stream
-// offsets [B][Hkv][mstride] uint32, candidate masks [B][Hkv][mstride][G] uint16, thresholds
-// [B][Hq] fp32, input pointers [3]
+// indexer workspace, in order: candidate streams (B*Hq*n_cap fp32), per-(head, page) records
+// {stream offset, candidate mask} [B][Hq][mstride] uint2, thresholds [B][Hq] fp32, input pointers [3]
 long topk_mstride(const Dims& d) { return ((long)d.max_pages + 7) & ~7L; }
 struct TopkLayout {
-    size_t cand, poff, pmask, tau, inputs, total;
+    size_t cand, prec, tau, inputs, total;
 };
 TopkLayout topk_layout(const Dims& d) {
     TopkLayout L;
     const size_t rows = (size_t)d.B * d.Hq;
-    const size_t recs = (size_t)d.B * d.Hkv * topk_mstride(d);
     L.cand = 0;
-    L.poff = align256(rows * d.n_cap * sizeof(float));
-    L.pmask = L.poff + align256(recs * sizeof(uint32_t));
-    L.tau = L.pmask + align256(recs * d.G * sizeof(uint16_t));
+    L.prec = align256(rows * d.n_cap * sizeof(float));
+    L.tau = L.prec + align256(rows * topk_mstride(d) * sizeof(uint2));
     L.inputs = L.tau + align256(rows * sizeof(float));
     L.total = L.inputs + align256(3 * sizeof(void*));
     return L;
@@ -237,8 +234,7 @@ sd_status topk_args(const sd_shape* shape, const void* q, const void* K, const i
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     if ((long)d.B * d.Hq * d.n_cap >= (1L << 32)) return SD_ERR_UNSUPPORTED;   // stream offsets are 32-bit
     a->cand = reinterpret_cast<float*>(ws + L.cand);
-    a->poff = reinterpret_cast<uint32_t*>(ws + L.poff);
-    a->pmask = reinterpret_cast<uint16_t*>(ws + L.pmask);
+    a->prec = reinterpret_cast<uint2*>(ws + L.prec);
     a->tau = reinterpret_cast<float*>(ws + L.tau);
     a->inputs = reinterpret_cast<const void**>(ws + L.inputs);
     a->mstride = (int)topk_mstride(d);

@@ -19,10 +19,10 @@ struct TopkArgs {
     const int32_t* k;
     int32_t* idx;
     float* cand;        // workspace, B*Hq*n_cap floats: candidate scores, one sequential stream per
-                        // score-pass warp; the candidates of unit (page p, kv head) are stored
-                        // head-major from cand[poff[...p]], each head's in position order
-    uint32_t* poff;     // workspace [B][Hkv][mstride]: where each (page, kv head) unit's candidates start
-    uint16_t* pmask;    // workspace [B][Hkv][mstride][G]: bit i = position p*16 + i of that head is a candidate
+                        // score-pass warp; the candidates of one (page, head) are consecutive, in
+                        // position order
+    uint2* prec;        // workspace [B][Hq][mstride]: per (head, page) {where its candidates start in
+                        // cand, 16-bit mask: bit i = position p*16 + i is a candidate}
     float* tau;         // workspace [B][Hq]: candidate threshold (scores >= tau are candidates;
                         // -inf: every position)
     const void** inputs;   // workspace [3]: q, K and page_table of the last score pass (the select
@@ -30,7 +30,7 @@ struct TopkArgs {
     int32_t* status;
     int B, Hq, Hkv, G, max_pages, num_pages, k_max;
     long n_cap;         // max_pages * page size: row stride of the score buffer
-    int mstride;        // pages per (request, kv head) record row (max_pages rounded up to 8)
+    int mstride;        // records per head row (max_pages rounded up to 8)
     int ccap;           // rows with N_b <= ccap take every position as a candidate
     int spp;            // pages per pipeline stage of the score pass
     int stages;         // pipeline depth of the score pass

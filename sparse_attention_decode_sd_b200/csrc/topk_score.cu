@@ -336,8 +336,7 @@ struct GroupCtx {
     int b = -1, kvh = -1, n = 0;
     uint32_t qf[NT][16];
     float tau[NT][2];       // candidate thresholds of head columns nt*8 + 2c + e (+inf past G)
-    uint32_t* poff_row;     // per page: where the unit's candidates start in the stream buffer
-    uint16_t* pmask_row;    // per page: G candidate masks
+    uint2* prec0;           // record row of head column 0 (the rows of the group's heads follow)
     __device__ __forceinline__ void load(const TopkArgs& a, int b_, int kvh_) {
         const int c = threadIdx.x & 3;
         load_q_frags_nat<NT>(a, b_, kvh_, qf);
@@ -348,9 +347,7 @@ struct GroupCtx {
                 const int col = nt * 8 + 2 * c + e;
                 tau[nt][e] = (col < a.G) ? __ldg(a.tau + (long)b_ * a.Hq + (long)kvh_ * a.G + col) : INFINITY;
             }
-        const long rec = ((long)b_ * a.Hkv + kvh_) * a.mstride;
-        poff_row = a.poff + rec;
-        pmask_row = a.pmask + rec * a.G;
+        prec0 = a.prec + ((long)b_ * a.Hq + (long)kvh_ * a.G) * a.mstride;
         n = a.lens[b_];
         b = b_;
         kvh = kvh_;
@@ -367,8 +364,8 @@ __device__ __forceinline__ void load_unit(uint32_t gbase, const uint32_t (&xo)[4
 
 // Scores NU units of one (request, kv head) group from their K fragments: 16 positions x G heads
 // each, two accumulation chains per unit.  Then appends each unit's candidates (scores >= tau) to the
-// warp's stream at `so` -- head by head, each head's in position order -- and records where they
-// start and the page's 16-bit candidate mask per head.
+// warp's stream at `so` -- head by head, each head's in position order -- and records per head where
+// they start and the page's 16-bit candidate mask.
 template <int NT, int NU>
 __device__ __forceinline__ void score_units(const TopkArgs& a, const GroupCtx<NT>& x, const uint32_t (&A)[NU][8][4],
                                             const int (&p)[NU], uint32_t& so) {
@@ -422,12 +419,11 @@ __device__ __forceinline__ void score_units(const TopkArgs& a, const GroupCtx<NT
                 if (c0 & (1u << lane)) a.cand[start + __popc(c0 & lt)] = sc[nt][e][0];
                 if (c1 & (1u << lane)) a.cand[start + __popc(c0) + __popc(c1 & lt)] = sc[nt][e][1];
                 if (g == 0 && col < a.G)
-                    x.pmask_row[(long)p[u] * a.G + col] =
-                        (uint16_t)(gather_nibble_bits(m0[nt][e] >> c) | (gather_nibble_bits(m1[nt][e] >> c) << 8));
+                    x.prec0[(long)col * a.mstride + p[u]] =
+                        make_uint2(start, gather_nibble_bits(m0[nt][e] >> c) | (gather_nibble_bits(m1[nt][e] >> c) << 8));
             }
             pre_nt += __popc(m0[nt][0]) + __popc(m1[nt][0]) + __popc(m0[nt][1]) + __popc(m1[nt][1]);
         }
-        if (lane == 0) x.poff_row[p[u]] = so;
         so += pre_nt;
     }
 }

@@ -176,60 +176,81 @@ __device__ void select_exact(const Src& src, int take, int32_t* row, int* hist, 
     emit_selected(src, T, take - greater, take, row, scratch);
 }
 
-// The candidates of row (b, h) as the score pass left them.  Per page p of the row's KV head:
-// pmask[p][col] marks which of the page's 16 positions are candidates for head col = h mod G, and
-// the page's candidates of all G heads sit head by head from cand[poff[p]] on.  Thread t of the
-// block owns the pages [t*per, (t+1)*per) and visits its candidates in ascending position order,
-// so a block scan over per-thread counts orders the whole row.
+// The candidates of row (b, h) as the score pass left them: per page p, the record
+// rec[p] = {start, mask}, mask bit i marking position p*16 + i as a candidate, whose scores sit in
+// position order from cand[start] on.  Thread t of the block owns the pages [t*per, (t+1)*per)
+// (per even, so that records come two to a 16-byte load) and visits its candidates in ascending
+// position order, so a block scan over per-thread counts orders the whole row.
 struct StreamRow {
     const float* cand;
-    const uint32_t* poff;
-    const uint16_t* pmask;
-    int G, col;
+    const uint2* rec;
     uint32_t limit;   // floats in the stream buffer: a record pointing past it is skipped (it can only
                       // come from a score pass that stopped early, which reported that)
     int p0, p1;       // this thread's pages
     __device__ StreamRow(const TopkArgs& a, long bh, int n) {
-        const int b = (int)(bh / a.Hq), h = (int)(bh % a.Hq), kvh = h / a.G;
-        const long rec = ((long)b * a.Hkv + kvh) * a.mstride;
         cand = a.cand;
-        poff = a.poff + rec;
-        pmask = a.pmask + rec * a.G;
-        G = a.G;
-        col = h - kvh * a.G;
+        rec = a.prec + bh * a.mstride;
         limit = (uint32_t)((long)a.B * a.Hq * a.n_cap);
         const int np = (n + kPageSize - 1) / kPageSize;
-        const int per = (np + (int)blockDim.x - 1) / (int)blockDim.x;
+        const int per = (((np + (int)blockDim.x - 1) / (int)blockDim.x) + 1) & ~1;
         p0 = min(np, (int)threadIdx.x * per);
         p1 = min(np, p0 + per);
     }
-    __device__ __forceinline__ uint32_t mask(int p) const { return pmask[(long)p * G + col]; }
+    __device__ __forceinline__ uint32_t mask(int p) const { return rec[p].y; }
+    __device__ __forceinline__ uint32_t record_base(int p) const { return rec[p].x; }
+    // This thread's candidate count (records loaded 16 at a time, all in flight together).
     __device__ __forceinline__ int count() const {
         int c = 0;
-        for (int p = p0; p < p1; ++p) c += __popc(mask(p));
+        for (int pb = p0; pb < p1; pb += 16) {
+#pragma unroll
+            for (int i = 0; i < 16; i += 2) {
+                if (pb + i + 1 < p1) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(rec + pb + i);
+                    c += __popc(v.y) + __popc(v.w);
+                } else if (pb + i < p1) {
+                    c += __popc(mask(pb + i));
+                }
+            }
+        }
         return c;
+    }
+    // Writes this thread's candidates in position order from slot `off` on: the position to pos[] and
+    // the candidate's index in the stream buffer to idx[] (0xffffffff for a record that points past
+    // the buffer).  Records are loaded 8 pages at a time.
+    __device__ __forceinline__ void stage(int off, uint32_t* idx, int* pos) const {
+        for (int pb = p0; pb < p1; pb += 8) {
+            uint2 r[8];
+#pragma unroll
+            for (int i = 0; i < 8; i += 2) {
+                if (pb + i + 1 < p1) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(rec + pb + i);
+                    r[i] = make_uint2(v.x, v.y);
+                    r[i + 1] = make_uint2(v.z, v.w);
+                } else {
+                    r[i] = (pb + i < p1) ? rec[pb + i] : make_uint2(0u, 0u);
+                    r[i + 1] = make_uint2(0u, 0u);
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                uint32_t mm = r[i].y;
+                const bool inside = (unsigned long)r[i].x + __popc(mm) <= limit;
+                for (uint32_t k = 0; mm; ++k) {
+                    const int bit = __ffs(mm) - 1;
+                    mm &= mm - 1u;
+                    idx[off] = inside ? r[i].x + k : 0xffffffffu;
+                    pos[off] = (pb + i) * kPageSize + bit;
+                    ++off;
+                }
+            }
+        }
     }
     template <class F>
     __device__ __forceinline__ void for_each(F f) const {
         for (int p = p0; p < p1; ++p) {
             uint32_t m = mask(p);
             if (m == 0u) continue;
-            uint32_t base = poff[p];
-            if ((G & 7) == 0) {   // records of 16-byte multiples: masks of the heads before col by vector
-                const uint4* r = reinterpret_cast<const uint4*>(pmask + (long)p * G);
-                for (int q = 0; q * 8 < col; ++q) {
-                    const uint4 v = r[q];
-                    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-                    const int below = min(8, col - q * 8);   // masks of this vector before col
-#pragma unroll
-                    for (int t = 0; t < 4; ++t) {
-                        const int nbits = min(32, max(0, 16 * (below - 2 * t)));
-                        base += __popc(nbits >= 32 ? w[t] : (w[t] & ((1u << nbits) - 1u)));
-                    }
-                }
-            } else {
-                for (int hh = 0; hh < col; ++hh) base += __popc((uint32_t)pmask[(long)p * G + hh]);
-            }
+            const uint32_t base = record_base(p);
             if ((unsigned long)base + __popc(m) > limit) continue;
             const float* sp = cand + base;
             for (int i = 0; m; ++i) {
@@ -355,12 +376,14 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(TopkArgs a) {
         __syncthreads();
         select_masked(RecomputedRow(a, bh, n, qs), take, row, hist, scratch, s_sel);
     } else if (total <= a.cap) {
-        // the usual case: the candidates, in position order, into shared memory
-        src.for_each([&](uint32_t key, int pos) {
-            lkey[off] = key;
-            lpos[off] = pos;
-            ++off;
-        });
+        // the usual case: the candidates, in position order, into shared memory -- positions and
+        // stream indices first, then every thread gathers scores (independent loads)
+        src.stage(off, lkey, lpos);
+        __syncthreads();
+        for (int j = tid; j < total; j += nthr) {
+            const uint32_t ix = lkey[j];
+            lkey[j] = ix < src.limit ? float_key(a.cand[ix]) : 0u;
+        }
         __syncthreads();
         select_exact(SharedKeys{lkey, lpos, total}, take, row, hist, scratch, s_sel);
     } else {

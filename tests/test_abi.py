@@ -71,9 +71,8 @@ def test_workspace_sizes(lib):
     topk = sdb.sd_workspace_size(s, sdb.SD_OP_TOPK)
     rows = 4 * 64
     scores = rows * 8192 * 16 * 4                          # fp32 candidate streams, B*Hq*n_cap
-    recs = 4 * 8 * 8192                                    # (request, kv head, page) records
-    small = recs * 4 + recs * 8 * 2 + rows * 4 + 3 * 8     # stream offsets, masks per head, thresholds, pointers
-    assert scores + small <= topk <= scores + small + 5 * 256
+    small = rows * 8192 * 8 + rows * 4 + 3 * 8             # (head, page) records, thresholds, pointers
+    assert scores + small <= topk <= scores + small + 4 * 256
     sparse = sdb.sd_workspace_size(s, sdb.SD_OP_SPARSE)
     assert sparse == sdb.sd_workspace_size(s, sdb.SD_OP_DENSE)
     slots = 4 * 64 * (8192 * 16 // 128 + 1)
