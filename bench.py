@@ -37,6 +37,8 @@ from sparse_attention_decode_sd_b200 import workloads as wl  # noqa: E402
 
 METRIC = "decode tokens/s and effective HBM GB/s (% of roofline) at 128K ctx, 50x sparsity"
 L2_FLUSH_BYTES = 512 << 20
+# kernels of one step: threshold, score pass, select; prep, union, decode, merge
+LAUNCHES_PER_STEP = 7
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -431,7 +433,7 @@ def run_ours(args):
         "e2e": {"value": tokens / (t_e2e / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": q_h.numel() * 2 + lens_h.numel() * 4 + k_h.numel() * 4,
                 "d2h_bytes_per_step": out_h.numel() * 4},
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)

@@ -15,7 +15,6 @@
 namespace sd {
 
 constexpr int kSelectThreads = 512;
-constexpr int kSelectItems = 4;   // consecutive elements per thread per tile of the exact emit
 
 // ---------------------------------------------------------------------------------------------
 // select
@@ -128,43 +127,31 @@ __device__ __forceinline__ void radix_find(const Src& src, int target, int* hist
 }
 
 // Writes the selected positions of src in ascending order to row[0..take): keys above T, plus the
-// first `quota` keys equal to T (ties go to the lower position).
+// first `quota` keys equal to T (ties go to the lower position).  Thread t takes a contiguous segment
+// of src; one block scan of its (greater, equal) counts, packed in one int, places its output.
 template <class Src>
 __device__ void emit_selected(const Src& src, uint32_t T, int quota, int take, int32_t* row, int* scratch) {
     const int tid = threadIdx.x, nthr = blockDim.x;
     const int n = src.size();
-    int out_base = 0, eq_base = 0;
-    for (int j0 = 0; j0 < n; j0 += nthr * kSelectItems) {
-        const int j = j0 + tid * kSelectItems;
-        uint32_t key[kSelectItems];
-        int eqc = 0;
-#pragma unroll
-        for (int e = 0; e < kSelectItems; ++e) {
-            key[e] = (j + e < n) ? src.key(j + e) : 0u;
-            eqc += (j + e < n && key[e] == T);
+    const int per = (n + nthr - 1) / nthr;
+    const int j0 = min(n, tid * per), j1 = min(n, j0 + per);
+    int gt = 0, eq = 0;
+    for (int j = j0; j < j1; ++j) {
+        const uint32_t key = src.key(j);
+        gt += key > T;
+        eq += key == T;
+    }
+    int tot;
+    const int before = block_exclusive_scan((eq << 16) | gt, scratch, &tot);   // counts < 2^15 each
+    int eq_before = before >> 16;
+    int w = (before & 0xffff) + min(eq_before, quota);
+    for (int j = j0; j < j1; ++j) {
+        const uint32_t key = src.key(j);
+        const bool keep = key > T || (key == T && eq_before++ < quota);
+        if (keep) {
+            if (w < take) row[w] = src.pos(j);
+            ++w;
         }
-        int eq_tot;
-        int eq_rank = eq_base + block_exclusive_scan(eqc, scratch, &eq_tot);
-        bool keep[kSelectItems];
-        int kc = 0;
-#pragma unroll
-        for (int e = 0; e < kSelectItems; ++e) {
-            const bool valid = j + e < n;
-            const bool eq = valid && key[e] == T;
-            keep[e] = valid && (key[e] > T || (eq && eq_rank < quota));
-            eq_rank += eq;
-            kc += keep[e];
-        }
-        int k_tot;
-        int w = out_base + block_exclusive_scan(kc, scratch, &k_tot);
-#pragma unroll
-        for (int e = 0; e < kSelectItems; ++e)
-            if (keep[e]) {
-                if (w < take) row[w] = src.pos(j + e);
-                ++w;
-            }
-        out_base += k_tot;
-        eq_base += eq_tot;
     }
 }
 
@@ -178,85 +165,100 @@ __device__ void select_exact(const Src& src, int take, int32_t* row, int* hist, 
 
 // The candidates of row (b, h) as the score pass left them: per page p, the record
 // rec[p] = {start, mask}, mask bit i marking position p*16 + i as a candidate, whose scores sit in
-// position order from cand[start] on.  Thread t of the block owns the pages [t*per, (t+1)*per)
-// (per even, so that records come two to a 16-byte load) and visits its candidates in ascending
-// position order, so a block scan over per-thread counts orders the whole row.
+// position order from cand[start] on.  The row's pages are taken in chunks of 16 * blockDim.x: in a
+// chunk, warp w owns 512 consecutive pages, read in 8 rounds of 64 with lane l holding pages
+// 2l and 2l + 1 of the round (one 16-byte load, coalesced across the warp).  Position order is
+// (warp, round, lane, record), which warp scans per round and a block scan over warps reproduce.
+constexpr int kRecsPerThread = 16;
+constexpr int kRounds = kRecsPerThread / 2;
 struct StreamRow {
     const float* cand;
     const uint2* rec;
     uint32_t limit;   // floats in the stream buffer: a record pointing past it is skipped (it can only
                       // come from a score pass that stopped early, which reported that)
-    int p0, p1;       // this thread's pages
+    int np;           // pages of the row
     __device__ StreamRow(const TopkArgs& a, long bh, int n) {
         cand = a.cand;
         rec = a.prec + bh * a.mstride;
         limit = (uint32_t)((long)a.B * a.Hq * a.n_cap);
-        const int np = (n + kPageSize - 1) / kPageSize;
-        const int per = (((np + (int)blockDim.x - 1) / (int)blockDim.x) + 1) & ~1;
-        p0 = min(np, (int)threadIdx.x * per);
-        p1 = min(np, p0 + per);
+        np = (n + kPageSize - 1) / kPageSize;
     }
-    __device__ __forceinline__ uint32_t mask(int p) const { return rec[p].y; }
-    __device__ __forceinline__ uint32_t record_base(int p) const { return rec[p].x; }
-    // This thread's candidate count (records loaded 16 at a time, all in flight together).
-    __device__ __forceinline__ int count() const {
-        int c = 0;
-        for (int pb = p0; pb < p1; pb += 16) {
+    __device__ __forceinline__ int chunks() const {
+        const int cp = kRecsPerThread * (int)blockDim.x;
+        return (np + cp - 1) / cp;
+    }
+    // first page of this lane's pair in round i of chunk ci
+    __device__ __forceinline__ int page_of(int ci, int i) const {
+        const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+        return ci * kRecsPerThread * (int)blockDim.x + warp * 32 * kRecsPerThread + i * 64 + 2 * lane;
+    }
+    // This lane's records of chunk ci, all loads in flight together (pages past the row read as empty).
+    __device__ __forceinline__ void load(int ci, uint2 (&r)[kRecsPerThread]) const {
+        uint4 v[kRounds];
 #pragma unroll
-            for (int i = 0; i < 16; i += 2) {
-                if (pb + i + 1 < p1) {
-                    const uint4 v = *reinterpret_cast<const uint4*>(rec + pb + i);
-                    c += __popc(v.y) + __popc(v.w);
-                } else if (pb + i < p1) {
-                    c += __popc(mask(pb + i));
-                }
-            }
+        for (int i = 0; i < kRounds; ++i) {
+            // the page index is even, and a row holds mstride >= np records with mstride a multiple of
+            // 8, so the pair lies in the row whenever its first page does; past the row read pair 0
+            const int p = page_of(ci, i);
+            v[i] = __ldg(reinterpret_cast<const uint4*>(rec + (p < np ? p : 0)));
         }
-        return c;
+#pragma unroll
+        for (int i = 0; i < kRounds; ++i) {
+            const int p = page_of(ci, i);
+            r[2 * i] = p < np ? make_uint2(v[i].x, v[i].y) : make_uint2(0u, 0u);
+            r[2 * i + 1] = p + 1 < np ? make_uint2(v[i].z, v[i].w) : make_uint2(0u, 0u);
+        }
     }
-    // Writes this thread's candidates in position order from slot `off` on: the position to pos[] and
-    // the candidate's index in the stream buffer to idx[] (0xffffffff for a record that points past
-    // the buffer).  Records are loaded 8 pages at a time.
-    __device__ __forceinline__ void stage(int off, uint32_t* idx, int* pos) const {
-        for (int pb = p0; pb < p1; pb += 8) {
-            uint2 r[8];
+    // Writes the candidates of records r (this lane's pages of chunk ci) in position order, the warp
+    // starting at slot `wbase`: the position to pos[] and the candidate's index in the stream buffer to
+    // idx[] (0xffffffff for a record that points past the buffer).  Every lane of the warp must call.
+    __device__ __forceinline__ void stage(int ci, const uint2 (&r)[kRecsPerThread], int wbase, uint32_t* idx,
+                                          int* pos) const {
+        const int lane = threadIdx.x & 31;
 #pragma unroll
-            for (int i = 0; i < 8; i += 2) {
-                if (pb + i + 1 < p1) {
-                    const uint4 v = *reinterpret_cast<const uint4*>(rec + pb + i);
-                    r[i] = make_uint2(v.x, v.y);
-                    r[i + 1] = make_uint2(v.z, v.w);
-                } else {
-                    r[i] = (pb + i < p1) ? rec[pb + i] : make_uint2(0u, 0u);
-                    r[i + 1] = make_uint2(0u, 0u);
-                }
+        for (int i = 0; i < kRounds; ++i) {
+            const int c = __popc(r[2 * i].y) + __popc(r[2 * i + 1].y);
+            int incl = c;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int t = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += t;
             }
+            int off = wbase + incl - c;
+            wbase += __shfl_sync(0xffffffffu, incl, 31);
+            const int p = page_of(ci, i);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                uint32_t mm = r[i].y;
-                const bool inside = (unsigned long)r[i].x + __popc(mm) <= limit;
+            for (int h = 0; h < 2; ++h) {
+                uint32_t mm = r[2 * i + h].y;
+                const uint32_t start = r[2 * i + h].x;
+                const bool inside = (unsigned long)start + __popc(mm) <= limit;
                 for (uint32_t k = 0; mm; ++k) {
                     const int bit = __ffs(mm) - 1;
                     mm &= mm - 1u;
-                    idx[off] = inside ? r[i].x + k : 0xffffffffu;
-                    pos[off] = (pb + i) * kPageSize + bit;
+                    idx[off] = inside ? start + k : 0xffffffffu;
+                    pos[off] = (p + h) * kPageSize + bit;
                     ++off;
                 }
             }
         }
     }
+    // Candidates of a thread-contiguous partition of the row (thread t: pages [t*per, (t+1)*per)), in
+    // position order, so that block scans over per-thread counts order the row -- for the passes that
+    // read the candidates from global memory.
     template <class F>
     __device__ __forceinline__ void for_each(F f) const {
+        const int per = (np + (int)blockDim.x - 1) / (int)blockDim.x;
+        const int p0 = min(np, (int)threadIdx.x * per), p1 = min(np, p0 + per);
         for (int p = p0; p < p1; ++p) {
-            uint32_t m = mask(p);
+            uint32_t m = rec[p].y;
             if (m == 0u) continue;
-            const uint32_t base = record_base(p);
+            const uint32_t base = rec[p].x;
             if ((unsigned long)base + __popc(m) > limit) continue;
             const float* sp = cand + base;
-            for (int i = 0; m; ++i) {
+            for (int k = 0; m; ++k) {
                 const int bit = __ffs(m) - 1;
                 m &= m - 1u;
-                f(float_key(sp[i]), p * kPageSize + bit);
+                f(float_key(sp[k]), p * kPageSize + bit);
             }
         }
     }
@@ -339,7 +341,7 @@ __device__ void select_masked(const Src& src, int take, int32_t* row, int* hist,
     });
 }
 
-__global__ void __launch_bounds__(kSelectThreads) select_kernel(TopkArgs a) {
+__global__ void __launch_bounds__(kSelectThreads, 2) select_kernel(TopkArgs a) {
     extern __shared__ __align__(1024) uint8_t smem[];
     int* hist = reinterpret_cast<int*>(smem);   // [4096]
     int* scratch = hist + 4096;                  // [40]
@@ -365,9 +367,23 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(TopkArgs a) {
         return;
     }
     StreamRow src(a, bh, n);
-    const int cnt = src.count();
-    int total;
-    int off = block_exclusive_scan(cnt, scratch, &total);
+    // Candidates chunk by chunk (one chunk up to 131072 positions): counted, and staged into shared
+    // memory in position order -- positions and stream indices -- while they fit.
+    int total = 0;
+    for (int ci = 0; ci < src.chunks(); ++ci) {
+        uint2 r[kRecsPerThread];
+        src.load(ci, r);
+        int cnt = 0;
+#pragma unroll
+        for (int i = 0; i < kRecsPerThread; ++i) cnt += __popc(r[i].y);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);   // the warp's count
+        int ctot;
+        const int wb = block_exclusive_scan((tid & 31) == 0 ? cnt : 0, scratch, &ctot);
+        const int wbase = total + __shfl_sync(0xffffffffu, wb, 0);   // candidates of the earlier warps
+        if (total + ctot <= a.cap) src.stage(ci, r, wbase, lkey, lpos);
+        total += ctot;
+    }
     if (total < take) {
         // the threshold admitted fewer candidates than k: select from scores recomputed on the fly
         float* qs = reinterpret_cast<float*>(lkey);
@@ -376,13 +392,23 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(TopkArgs a) {
         __syncthreads();
         select_masked(RecomputedRow(a, bh, n, qs), take, row, hist, scratch, s_sel);
     } else if (total <= a.cap) {
-        // the usual case: the candidates, in position order, into shared memory -- positions and
-        // stream indices first, then every thread gathers scores (independent loads)
-        src.stage(off, lkey, lpos);
+        // the usual case: every thread gathers scores for the staged stream indices, four loads in flight
         __syncthreads();
-        for (int j = tid; j < total; j += nthr) {
-            const uint32_t ix = lkey[j];
-            lkey[j] = ix < src.limit ? float_key(a.cand[ix]) : 0u;
+        for (int j0 = tid; j0 < total; j0 += 4 * nthr) {
+            uint32_t ix[4];
+            float v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int j = j0 + u * nthr;
+                ix[u] = j < total ? lkey[j] : 0xffffffffu;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) v[u] = ix[u] < src.limit ? __ldg(a.cand + ix[u]) : 0.f;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int j = j0 + u * nthr;
+                if (j < total) lkey[j] = ix[u] < src.limit ? float_key(v[u]) : 0u;
+            }
         }
         __syncthreads();
         select_exact(SharedKeys{lkey, lpos, total}, take, row, hist, scratch, s_sel);
