@@ -105,6 +105,36 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const void* tmap, int x, 
         : "memory");
 }
 
+// The same with an L2 cache-eviction policy (from l2_policy_*) for the loaded lines.
+__device__ __forceinline__ void tma_load_4d_hint(void* dst, const void* tmap, int x, int y, int z, int w, uint64_t* bar,
+                                                 uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, "
+        "{%2, %3, %4, %5}], [%6], %7;\n" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_addr(bar)), "l"(policy)
+        : "memory");
+}
+
+// L2 cache-eviction policies covering every access they are attached to: lines to let go first
+// (read-once streams) and lines to keep (data the next kernel reads).
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;\n" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;\n" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ void st_hint(float* p, float v, uint64_t policy) {
+    asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;\n" ::"l"(p), "f"(v), "l"(policy) : "memory");
+}
+__device__ __forceinline__ void st_hint(uint2* p, uint2 v, uint64_t policy) {
+    asm volatile("st.global.L2::cache_hint.v2.u32 [%0], {%1, %2}, %3;\n" ::"l"(p), "r"(v.x), "r"(v.y), "l"(policy)
+                 : "memory");
+}
+
 // ---------------------------------------------------------------------------------------------
 // Thread-block clusters: rank, cluster-wide barrier, distributed shared memory stores.
 // ---------------------------------------------------------------------------------------------

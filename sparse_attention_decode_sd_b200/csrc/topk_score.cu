@@ -310,6 +310,7 @@ struct StageIssuer {
     long t0, t1;
     int stage_bytes, page_bytes;
     int b;   // request cursor (stages are issued in order)
+    uint64_t stream_policy;   // K is read once here: its lines go first from L2
     __device__ void issue(long st, int slot) {
         const long tb = t0 + st * a->spp;
         const int np = (int)min((long)a->spp, t1 - tb);
@@ -324,8 +325,8 @@ struct StageIssuer {
                 page = 0;   // keep the transaction count whole; the scores of this page are void
             }
             uint8_t* dst = data + (size_t)slot * stage_bytes + (size_t)i * page_bytes;
-            tma_load_4d(dst, tmap, 0, 0, 0, page, &full[slot]);
-            tma_load_4d(dst + page_bytes / 2, tmap, 64, 0, 0, page, &full[slot]);
+            tma_load_4d_hint(dst, tmap, 0, 0, 0, page, &full[slot], stream_policy);
+            tma_load_4d_hint(dst + page_bytes / 2, tmap, 64, 0, 0, page, &full[slot], stream_policy);
         }
     }
 };
@@ -370,6 +371,7 @@ template <int NT, int NU>
 __device__ __forceinline__ void score_units(const TopkArgs& a, const GroupCtx<NT>& x, const uint32_t (&A)[NU][8][4],
                                             const int (&p)[NU], uint32_t& so) {
     const int lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
+    const uint64_t keep = l2_policy_evict_last();   // the select step reads candidates and records next
     const uint32_t lt = (1u << lane) - 1u;
     const uint32_t mc = 0x11111111u << c;                // lanes holding this lane's two head columns
     const uint32_t mlt = 0x11111111u * ((1u << c) - 1u);  // lanes holding the columns before them
@@ -416,11 +418,12 @@ __device__ __forceinline__ void score_units(const TopkArgs& a, const GroupCtx<NT
                 const int col = nt * 8 + 2 * c + e;
                 const uint32_t c0 = m0[nt][e] & mc, c1 = m1[nt][e] & mc;
                 const uint32_t start = so + pre_nt + before + (e ? __popc(m0[nt][0] & mc) + __popc(m1[nt][0] & mc) : 0u);
-                if (c0 & (1u << lane)) a.cand[start + __popc(c0 & lt)] = sc[nt][e][0];
-                if (c1 & (1u << lane)) a.cand[start + __popc(c0) + __popc(c1 & lt)] = sc[nt][e][1];
+                if (c0 & (1u << lane)) st_hint(a.cand + start + __popc(c0 & lt), sc[nt][e][0], keep);
+                if (c1 & (1u << lane)) st_hint(a.cand + start + __popc(c0) + __popc(c1 & lt), sc[nt][e][1], keep);
                 if (g == 0 && col < a.G)
-                    x.prec0[(long)col * a.mstride + p[u]] =
-                        make_uint2(start, gather_nibble_bits(m0[nt][e] >> c) | (gather_nibble_bits(m1[nt][e] >> c) << 8));
+                    st_hint(x.prec0 + (long)col * a.mstride + p[u],
+                            make_uint2(start, gather_nibble_bits(m0[nt][e] >> c) | (gather_nibble_bits(m1[nt][e] >> c) << 8)),
+                            keep);
             }
             pre_nt += __popc(m0[nt][0]) + __popc(m1[nt][0]) + __popc(m0[nt][1]) + __popc(m1[nt][1]);
         }
@@ -564,7 +567,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_pass_kernel(TopkArgs a
     if (warp == kScoreConsumerWarps) {
         // ---------------- producer: one thread issues the tensor copies ----------------
         if (lane != 0) return;
-        StageIssuer is{&a, &tmap, prefix, data, full, t0, t1, stage_bytes, page_bytes, locate_request(prefix, a.B, t0)};
+        StageIssuer is{&a, &tmap, prefix, data, full, t0, t1, stage_bytes, page_bytes, locate_request(prefix, a.B, t0),
+                       l2_policy_evict_first()};
         long issued = 0;
         int slot = 0;
         uint32_t phase = 0;   // parity of the release the slot's next refill waits for

@@ -310,8 +310,10 @@ struct RecomputedRow {
 // Selection straight from a source visited with for_each in thread-ordered position order (any
 // number of candidates): radix select, then the ascending positions through two block scans (ties
 // first, then the selected).
+// (Not inlined: these paths are rare, and their registers stay out of the usual path's budget.)
 template <class Src>
-__device__ void select_masked(const Src& src, int take, int32_t* row, int* hist, int* scratch, int* s_sel) {
+__device__ __noinline__ void select_masked(const Src& src, int take, int32_t* row, int* hist, int* scratch,
+                                          int* s_sel) {
     uint32_t T;
     int greater;
     radix_select([&](auto f) { src.for_each([&](uint32_t key, int) { f(key); }); }, take, hist, scratch, s_sel, &T,
@@ -371,17 +373,24 @@ __global__ void __launch_bounds__(kSelectThreads, 2) select_kernel(TopkArgs a) {
     // memory in position order -- positions and stream indices -- while they fit.
     int total = 0;
     for (int ci = 0; ci < src.chunks(); ++ci) {
-        uint2 r[kRecsPerThread];
-        src.load(ci, r);
-        int cnt = 0;
+        int cnt;
+        {
+            uint2 r[kRecsPerThread];
+            src.load(ci, r);
+            cnt = 0;
 #pragma unroll
-        for (int i = 0; i < kRecsPerThread; ++i) cnt += __popc(r[i].y);
+            for (int i = 0; i < kRecsPerThread; ++i) cnt += __popc(r[i].y);
+        }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);   // the warp's count
         int ctot;
         const int wb = block_exclusive_scan((tid & 31) == 0 ? cnt : 0, scratch, &ctot);
         const int wbase = total + __shfl_sync(0xffffffffu, wb, 0);   // candidates of the earlier warps
-        if (total + ctot <= a.cap) src.stage(ci, r, wbase, lkey, lpos);
+        if (total + ctot <= a.cap) {
+            uint2 r[kRecsPerThread];
+            src.load(ci, r);   // again, from L1: cheaper than keeping 32 registers across the scan
+            src.stage(ci, r, wbase, lkey, lpos);
+        }
         total += ctot;
     }
     if (total < take) {
