@@ -61,9 +61,9 @@ def source_hash(*names):
 
 
 KERNEL_SOURCES = {
-    "score_pass_kernel": ("topk_score.cu", "common.cuh"),
-    "select_kernel": ("topk_select.cu", "common.cuh"),
-    "decode_kernel": ("sparse_decode.cu", "common.cuh"),
+    "score_pass_kernel": ("topk_score.cu", "common.cuh", "kernels.h"),
+    "select_kernel": ("topk_select.cu", "common.cuh", "kernels.h"),
+    "decode_kernel": ("sparse_decode.cu", "common.cuh", "kernels.h"),
 }
 
 
