@@ -241,9 +241,13 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* scratch, int* to
 // then waits until the previous kernel has completed and its memory is visible, before touching
 // anything.  (Both instructions are no-ops when a kernel was launched without the attribute.)
 // ---------------------------------------------------------------------------------------------
-__device__ __forceinline__ void pdl_enter() {
+__device__ __forceinline__ void pdl_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
-    asm volatile("griddepcontrol.wait;\n" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void pdl_enter() {
+    pdl_launch_dependents();
+    pdl_wait();
 }
 
 template <typename... KArgs, typename... Args>

@@ -28,7 +28,7 @@
 namespace sd {
 
 constexpr int kScoreConsumerWarps = 8;   // plus one producer warp that issues the copies
-constexpr int kThresholdWarps = 8;
+constexpr int kThresholdWarps = 4;   // 4 warps: a threshold CTA fits beside a score-pass CTA
 constexpr int kScoreThreads = (kScoreConsumerWarps + 1) * 32;
 
 // Pages request b contributes to the score pass: every page of N_b, unless no selection is needed
@@ -228,7 +228,10 @@ __global__ void __cluster_dims__(kThresholdCluster, 1, 1) __launch_bounds__(kThr
     uint16_t* skey = reinterpret_cast<uint16_t*>(smem);                // [NT][kSample]: columns r, r + 8
     int* hist = reinterpret_cast<int*>(skey + NT * kSample);           // [warps][256]
     int* s_res = hist + 256 * kThresholdWarps;                         // [8]
-    pdl_enter();
+    // Wait for the work before this kernel first, then let the score pass launch: the score pass starts
+    // streaming K at once, which is safe only once everything before this kernel has completed.
+    pdl_wait();
+    pdl_launch_dependents();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, g = lane >> 2, c = lane & 3;
     const uint32_t rank = cluster_ctarank();
     const int grp = blockIdx.x / kThresholdCluster;
@@ -249,38 +252,43 @@ __global__ void __cluster_dims__(kThresholdCluster, 1, 1) __launch_bounds__(kThr
     load_q_frags<NT>(a, b, kvh, qf);
     const int32_t* ptrow = a.page_table + (long)b * a.max_pages;
     const uint32_t skey_s = smem_addr(skey);
-    // two tiles per warp, with all four K-row loads of a warp in flight together
+    // kTilesPerWarp tiles per warp, two at a time with all four K-row loads of a pair in flight together
     constexpr int kTilesPerCta = kSample / 16 / kThresholdCluster;
-    uint32_t R[2][2][16];
+    constexpr int kTilesPerWarp = kTilesPerCta / kThresholdWarps;
+    static_assert(kTilesPerWarp % 2 == 0, "tiles go in pairs");
+#pragma unroll 1
+    for (int t0 = 0; t0 < kTilesPerWarp; t0 += 2) {
+        uint32_t R[2][2][16];
 #pragma unroll
-    for (int t = 0; t < 2; ++t)
+        for (int t = 0; t < 2; ++t)
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            const int tile = (int)rank * kTilesPerCta + warp + kThresholdWarps * t;
-            const int i = tile * 16 + g + 8 * half;
-            const int p = (int)(((long)i * n) / kSample);
-            int page = __ldg(ptrow + p / kPageSize);
-            if (page < 0 || page >= a.num_pages) page = 0;   // reported by the score pass
-            load_k_row_global(a.K + (((long)page * kPageSize + (p % kPageSize)) * a.Hkv + kvh) * kHeadDim, c,
-                              R[t][half]);
-        }
-#pragma unroll
-    for (int t = 0; t < 2; ++t) {
-        const int tile = (int)rank * kTilesPerCta + warp + kThresholdWarps * t;
-        float acc[NT][4];
-        score_tile<NT>(R[t][0], R[t][1], qf, acc);
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int col = nt * 8 + 2 * c + e;
-                if (col < a.G) {
-                    const uint32_t dst = map_shared_rank(skey_s, (uint32_t)(col & 7)) +
-                                         (uint32_t)(((col >> 3) * kSample + tile * 16 + g) * 2);
-                    st_cluster_u16(dst, (uint16_t)(float_key(acc[nt][e]) >> 16));
-                    st_cluster_u16(dst + 16u, (uint16_t)(float_key(acc[nt][2 + e]) >> 16));
-                }
+            for (int half = 0; half < 2; ++half) {
+                const int tile = (int)rank * kTilesPerCta + warp + kThresholdWarps * (t0 + t);
+                const int i = tile * 16 + g + 8 * half;
+                const int p = (int)(((long)i * n) / kSample);
+                int page = __ldg(ptrow + p / kPageSize);
+                if (page < 0 || page >= a.num_pages) page = 0;   // reported by the score pass
+                load_k_row_global(a.K + (((long)page * kPageSize + (p % kPageSize)) * a.Hkv + kvh) * kHeadDim, c,
+                                  R[t][half]);
             }
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+            const int tile = (int)rank * kTilesPerCta + warp + kThresholdWarps * (t0 + t);
+            float acc[NT][4];
+            score_tile<NT>(R[t][0], R[t][1], qf, acc);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int col = nt * 8 + 2 * c + e;
+                    if (col < a.G) {
+                        const uint32_t dst = map_shared_rank(skey_s, (uint32_t)(col & 7)) +
+                                             (uint32_t)(((col >> 3) * kSample + tile * 16 + g) * 2);
+                        st_cluster_u16(dst, (uint16_t)(float_key(acc[nt][e]) >> 16));
+                        st_cluster_u16(dst + 16u, (uint16_t)(float_key(acc[nt][2 + e]) >> 16));
+                    }
+                }
+        }
     }
     cluster_sync_all();   // every sample key is in place
     const int kth = sample_rank(kb, n);
@@ -340,6 +348,7 @@ struct GroupCtx {
     uint2* prec0;           // record row of head column 0 (the rows of the group's heads follow)
     __device__ __forceinline__ void load(const TopkArgs& a, int b_, int kvh_) {
         const int c = threadIdx.x & 3;
+        pdl_wait();   // the thresholds come from the kernel before this one (returns at once after the first)
         load_q_frags_nat<NT>(a, b_, kvh_, qf);
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
@@ -519,9 +528,12 @@ __device__ __forceinline__ void consume(const TopkArgs& a, const uint8_t* data, 
 }
 
 template <int NT>
-__global__ void __launch_bounds__(kScoreThreads, 1) score_pass_kernel(TopkArgs a, const __grid_constant__ CUtensorMap tmap) {
+__device__ __forceinline__ void score_pass(const TopkArgs& a, const CUtensorMap& tmap) {
     extern __shared__ __align__(1024) uint8_t smem[];
-    pdl_enter();
+    // No wait here: the threshold kernel launched this grid only after the work before it had completed,
+    // so the inputs can be read at once and the K stream overlaps the threshold kernel.  Its output, the
+    // thresholds, is read after griddepcontrol.wait (GroupCtx::load).
+    pdl_launch_dependents();
     const int page_bytes = kPageSize * a.Hkv * kRowBytes;
     const int half_bytes = page_bytes / 2;
     const int stage_bytes = a.spp * page_bytes;
@@ -596,6 +608,19 @@ __global__ void __launch_bounds__(kScoreThreads, 1) score_pass_kernel(TopkArgs a
     // not it has a unit there, which keeps the arrival count of each release barrier fixed.  With
     // Hkv dividing 8, a warp always meets the same KV head.
     consume<NT>(a, data, full, empty, prefix, t0, t1, nst, half_bytes, stage_bytes, page_bytes);
+}
+
+// G <= 8.  At most 144 registers per thread: a threshold CTA (4 warps, <= 80 registers) then fits on
+// an SM beside a score-pass CTA -- also within each SM sub-partition's register file, which holds three
+// of the score pass's nine warps plus one threshold warp -- so the score pass starts streaming K while
+// the threshold kernel finishes.
+__global__ void __maxnreg__(144) score_pass_kernel_g8(TopkArgs a, const __grid_constant__ CUtensorMap tmap) {
+    score_pass<1>(a, tmap);
+}
+// 8 < G <= 16.
+__global__ void __launch_bounds__(kScoreThreads, 1) score_pass_kernel_g16(TopkArgs a,
+                                                                          const __grid_constant__ CUtensorMap tmap) {
+    score_pass<2>(a, tmap);
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -683,13 +708,13 @@ cudaError_t launch_score_pass(const TopkArgs& a, int grid, cudaStream_t stream) 
     if (e != cudaSuccess) return e;
     const size_t smem = score_pass_smem(a);
     if (a.G <= 8) {
-        e = cudaFuncSetAttribute(score_pass_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        e = cudaFuncSetAttribute(score_pass_kernel_g8, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        e = launch_pdl(score_pass_kernel<1>, dim3(grid), dim3(kScoreThreads), smem, stream, a, tmap);
+        e = launch_pdl(score_pass_kernel_g8, dim3(grid), dim3(kScoreThreads), smem, stream, a, tmap);
     } else {
-        e = cudaFuncSetAttribute(score_pass_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        e = cudaFuncSetAttribute(score_pass_kernel_g16, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        e = launch_pdl(score_pass_kernel<2>, dim3(grid), dim3(kScoreThreads), smem, stream, a, tmap);
+        e = launch_pdl(score_pass_kernel_g16, dim3(grid), dim3(kScoreThreads), smem, stream, a, tmap);
     }
     return e != cudaSuccess ? e : cudaGetLastError();
 }
