@@ -66,7 +66,10 @@ def _configure(lib):
     lib.oracle_topk.argtypes = [I] * 8 + [P, P, P, P, P, P]
     lib.oracle_attend.argtypes = [I] * 8 + [P, P, P, P, P, P, P]
     lib.oracle_dense.argtypes = [I] * 7 + [P, P, P, P, P, P]
-    for f in (lib.oracle_scores, lib.oracle_topk, lib.oracle_attend, lib.oracle_dense):
+    lib.oracle_quest_scores.argtypes = [I] * 7 + [P, P, P, P, I, I, P]
+    lib.oracle_quest_topk.argtypes = [I] * 8 + [P, P, P, P, P, P]
+    for f in (lib.oracle_scores, lib.oracle_topk, lib.oracle_attend, lib.oracle_dense, lib.oracle_quest_scores,
+              lib.oracle_quest_topk):
         f.restype = ctypes.c_int
     lib.oracle_num_threads.restype = ctypes.c_int
     return lib
@@ -166,3 +169,27 @@ def dense(shape: dict, q, K, V, page_table, lens) -> np.ndarray:
     _check(_load().oracle_dense(B, Hq, Hkv, d, P, max_pages, num_pages, _p(qa), _p(Ka), _p(Va), _p(pt), _p(ln),
                                 _p(out)), "dense")
     return out
+
+
+def quest_scores(shape: dict, q, K, page_table, lens, b: int, h: int) -> np.ndarray:
+    """Quest page relevance r_j = sum_d max(q_d min_d, q_d max_d) of every page of (b, h)."""
+    B, Hq, Hkv, d, P, max_pages = _dims(shape)
+    qa, Ka, pt, ln = _u16(q), _u16(K), _i32(page_table), _i32(lens)
+    num_pages = Ka.size // (P * Hkv * d)
+    np_ = (int(ln[b]) + P - 1) // P
+    out = np.zeros(max(np_, 1), dtype=np.float64)
+    _check(_load().oracle_quest_scores(B, Hq, Hkv, d, P, max_pages, num_pages, _p(qa), _p(Ka), _p(pt), _p(ln),
+                                       int(b), int(h), _p(out)), "quest_scores")
+    return out[:np_]
+
+
+def quest_topk(shape: dict, q, K, page_table, lens, k, k_max: int | None = None) -> np.ndarray:
+    """Quest selection: positions of the current page plus the ceil(k_b / P) - 1 most relevant others."""
+    B, Hq, Hkv, d, P, max_pages = _dims(shape)
+    k_max = int(shape["k_max"] if k_max is None else k_max)
+    qa, Ka, pt, ln, ka = _u16(q), _u16(K), _i32(page_table), _i32(lens), _i32(k)
+    num_pages = Ka.size // (P * Hkv * d)
+    idx = np.full((B, Hq, max(k_max, 0)), -1, dtype=np.int32)
+    _check(_load().oracle_quest_topk(B, Hq, Hkv, d, P, max_pages, num_pages, k_max, _p(qa), _p(Ka), _p(pt),
+                                     _p(ln), _p(ka), _p(idx)), "quest_topk")
+    return idx

@@ -20,6 +20,15 @@
  *              -- SDPA restricted to the selected rows, softmax renormalised over S only
  *              (same SDPA formula; Fig. 1(a) "Sparse" mode reads only the k selected rows).
  *   dense      attend with S = all N_b positions (Fig. 1(a) "Dense" mode).
+ *   quest      the page-level approximate indexer Quest ("The Sparse Frontier" review (xllm),
+ *              sec. 7.1 "Quest" and Table 1; memory model Eq. 10): pages of P positions, each
+ *              represented per KV head by the per-dimension minimum and maximum of its keys;
+ *              per (b, h) the "most relevant" pages are kept, always including the page that holds
+ *              the current (last) position.  The pages do not spell out relevance; the reading
+ *              here is the largest q.k that any key inside the page's box [min, max] can reach,
+ *              r_j = sum_d max(q_d * min_d, q_d * max_d).  Budget: ceil(k_b / P) pages (the
+ *              current page plus the best others, ties to the lower page); the selection is
+ *              every position < N_b of the kept pages, ascending.
  *
  * Data layout read here (the paged KV cache the pages describe as a paged-KV backend,
  * "Inference-time context sparsity", sec. 1, "sparsity is usable for systems gains"):
@@ -251,6 +260,113 @@ int oracle_dense(int B, int Hq, int Hkv, int d, int P, int max_pages, int num_pa
             rc = attend_one(&s, q, K, V, page_table, b, h, n, sel, n, out + bh * (long)d);
         }
         free(sel);
+        if (rc < rc_all) rc_all = rc;
+    }
+    return rc_all;
+}
+
+/* Quest page representation of logical page j of request b, KV head kvh: the per-dimension minimum
+ * and maximum over the page's positions that exist (those < N_b), in double. */
+static int quest_box(const oshape* s, const uint16_t* K, const int32_t* page_table, int b, int kvh, int n, long j,
+                     double* mn, double* mx) {
+    long p0 = j * s->P, p1 = p0 + s->P;
+    if (p1 > n) p1 = n;
+    for (long p = p0; p < p1; ++p) {
+        const uint16_t* krow = cache_row(s, K, page_table, b, kvh, p);
+        if (!krow) return -2;
+        for (int e = 0; e < s->d; ++e) {
+            double v = bf16_to_double(krow[e]);
+            if (p == p0 || v < mn[e]) mn[e] = v;
+            if (p == p0 || v > mx[e]) mx[e] = v;
+        }
+    }
+    return 0;
+}
+
+/* r_j = sum_d max(q_d * min_d, q_d * max_d) for every page j < ceil(N_b / P) of (b, h). */
+static int quest_scores_one(const oshape* s, const uint16_t* q, const uint16_t* K, const int32_t* page_table,
+                            int b, int h, int n, double* out) {
+    int G = s->Hq / s->Hkv;
+    int kvh = h / G;
+    const uint16_t* qh = q + ((long)b * s->Hq + h) * s->d;
+    long np = ((long)n + s->P - 1) / s->P;
+    double* mn = (double*)malloc(sizeof(double) * (size_t)s->d);
+    double* mx = (double*)malloc(sizeof(double) * (size_t)s->d);
+    if (!mn || !mx) { free(mn); free(mx); return -4; }
+    int rc = 0;
+    for (long j = 0; j < np && rc == 0; ++j) {
+        rc = quest_box(s, K, page_table, b, kvh, n, j, mn, mx);
+        double r = 0.0;
+        for (int e = 0; e < s->d && rc == 0; ++e) {
+            double qe = bf16_to_double(qh[e]);
+            double lo = qe * mn[e], hi = qe * mx[e];
+            r += lo > hi ? lo : hi;
+        }
+        out[j] = r;
+    }
+    free(mn);
+    free(mx);
+    return rc;
+}
+
+int oracle_quest_scores(int B, int Hq, int Hkv, int d, int P, int max_pages, int num_pages,
+                        const uint16_t* q, const uint16_t* K, const int32_t* page_table, const int32_t* lens,
+                        int b, int h, double* out) {
+    oshape s = {B, Hq, Hkv, d, P, max_pages, 0, num_pages};
+    if (check_shape(&s) || b < 0 || b >= B || h < 0 || h >= Hq) return -1;
+    int n = req_len(&s, lens, b);
+    if (n < 0) return -1;
+    return quest_scores_one(&s, q, K, page_table, b, h, n, out);
+}
+
+/* Quest selection of one (b, h): the current page (the last one) plus the ceil(k_b / P) - 1 other
+ * pages with the largest r (ties to the lower page); all their positions < N_b, ascending, then -1. */
+static int quest_one(const oshape* s, const uint16_t* q, const uint16_t* K, const int32_t* page_table,
+                     int b, int h, int n, int kb, int32_t* idx_row) {
+    for (int i = 0; i < s->k_max; ++i) idx_row[i] = -1;
+    if (n <= 0) return 0;
+    long np = ((long)n + s->P - 1) / s->P;
+    long kp = ((long)kb + s->P - 1) / s->P;
+    if (kp > np) kp = np;
+    char* keep = (char*)calloc((size_t)np, 1);
+    double* r = (double*)malloc(sizeof(double) * (size_t)np);
+    scored* other = (scored*)malloc(sizeof(scored) * (size_t)np);
+    if (!keep || !r || !other) { free(keep); free(r); free(other); return -4; }
+    int rc = quest_scores_one(s, q, K, page_table, b, h, n, r);
+    if (rc == 0) {
+        keep[np - 1] = 1;   /* the page of the current position is always kept */
+        for (long j = 0; j + 1 < np; ++j) { other[j].s = r[j]; other[j].pos = (int32_t)j; }
+        qsort(other, (size_t)(np - 1), sizeof(scored), by_score_then_pos);
+        for (long t = 0; t + 1 < kp; ++t) keep[other[t].pos] = 1;
+        long w = 0;
+        for (long j = 0; j < np && rc == 0; ++j) {
+            if (!keep[j]) continue;
+            for (long p = j * s->P; p < (j + 1) * s->P && p < n; ++p) {
+                if (w >= s->k_max) { rc = -3; break; }
+                idx_row[w++] = (int32_t)p;
+            }
+        }
+    }
+    free(keep);
+    free(r);
+    free(other);
+    return rc;
+}
+
+int oracle_quest_topk(int B, int Hq, int Hkv, int d, int P, int max_pages, int num_pages, int k_max,
+                      const uint16_t* q, const uint16_t* K, const int32_t* page_table, const int32_t* lens,
+                      const int32_t* k, int32_t* idx) {
+    oshape s = {B, Hq, Hkv, d, P, max_pages, k_max, num_pages};
+    if (check_shape(&s)) return -1;
+    for (int b = 0; b < B; ++b) {
+        if (req_len(&s, lens, b) < 0) return -1;
+        if (k[b] < 1) return -1;
+    }
+    int rc_all = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(min : rc_all)
+    for (long bh = 0; bh < (long)B * Hq; ++bh) {
+        int b = (int)(bh / Hq), h = (int)(bh % Hq);
+        int rc = quest_one(&s, q, K, page_table, b, h, lens[b], k[b], idx + bh * (long)k_max);
         if (rc < rc_all) rc_all = rc;
     }
     return rc_all;

@@ -13,6 +13,7 @@ import pytest
 
 import oracle
 from tests import test_oracle as pins
+from tests import test_oracle_quest as quest_pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
 
@@ -34,6 +35,17 @@ MUTANTS = [
     ("one_row_short", "for (int i = 0; i < take; ++i) idx_row[i] = all[i].pos;",
      "for (int i = 0; i + 1 < take; ++i) idx_row[i] = all[i].pos;"),
     ("unsorted_output", "qsort(idx_row, (size_t)take, sizeof(int32_t), by_pos);", ""),
+    # Quest
+    ("quest_lower_bound_instead_of_upper", "r += lo > hi ? lo : hi;", "r += lo < hi ? lo : hi;"),
+    # (swapping min and max is not a mistake: the relevance is symmetric in them)
+    ("quest_max_only", "double lo = qe * mn[e], hi = qe * mx[e];", "double lo = qe * mx[e], hi = qe * mx[e];"),
+    ("quest_stale_slots_counted", "    if (p1 > n) p1 = n;\n", ""),
+    ("quest_current_page_dropped", "keep[np - 1] = 1;   /* the page of the current position is always kept */", ""),
+    ("quest_budget_rounds_down", "long kp = ((long)kb + s->P - 1) / s->P;", "long kp = (long)kb / s->P;"),
+    ("quest_current_page_outside_budget", "for (long t = 0; t + 1 < kp; ++t) keep[other[t].pos] = 1;",
+     "for (long t = 0; t < kp && t + 1 < np; ++t) keep[other[t].pos] = 1;"),
+    ("quest_first_dim_dropped", "for (int e = 0; e < s->d && rc == 0; ++e) {\n            double qe",
+     "for (int e = 1; e < s->d && rc == 0; ++e) {\n            double qe"),
 ]
 
 PINS = [
@@ -46,6 +58,12 @@ PINS = [
     pins.test_k1_returns_argmax_row,
     pins.test_two_rows_logistic_closed_form,
     pins.test_golden_uniform_average,
+    quest_pins.test_relevance_is_max_over_box_corners,
+    quest_pins.test_relevance_bounds_every_row_of_its_page,
+    quest_pins.test_current_page_always_kept,
+    quest_pins.test_ties_go_to_lower_page_and_budget_rounds_up,
+    quest_pins.test_partial_last_page_and_whole_cache_budget,
+    quest_pins.test_selection_is_the_most_relevant_pages,
 ]
 
 
