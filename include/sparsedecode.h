@@ -80,9 +80,10 @@ enum {
     SD_ERR_ORDER = 7          /* device: an idx row is not strictly ascending */
 };
 
-enum { SD_OP_TOPK = 1, SD_OP_SPARSE = 2, SD_OP_DENSE = 3 };
+enum { SD_OP_TOPK = 1, SD_OP_SPARSE = 2, SD_OP_DENSE = 3, SD_OP_QUEST = 4 };
 
-/* Bytes of workspace that operation `op` needs for `shape` (independent of the data and of the
+/* Bytes of workspace that operation `op` (SD_OP_TOPK, SD_OP_SPARSE, SD_OP_DENSE, SD_OP_QUEST) needs
+ * for `shape` (independent of the data and of the
  * device).  Returns SD_ERR_INVALID_ARG / SD_ERR_UNSUPPORTED for a shape the library rejects. */
 SD_API sd_status sd_workspace_size(const sd_shape* shape, int32_t op, size_t* bytes);
 
@@ -160,6 +161,36 @@ SD_API sd_status sd_dense_decode(const sd_shape* shape, const void* q, const voi
 SD_API sd_status sd_append_kv(const sd_shape* shape, void* K, void* V, const int32_t* page_table, int32_t* lens,
                        const void* k_new, const void* v_new, int32_t* k_sel, int32_t ratio,
                        int32_t* dev_status, void* stream);
+
+/* Quest, the page-level approximate indexer ("The Sparse Frontier" review, sec. 7.1 "Quest" and
+ * Table 1; its memory model is Eq. 10 there): pages of P = 16 positions, each represented per KV head
+ * by the per-dimension minimum and maximum of its keys ("boxes"); per decode query and query head the
+ * most relevant pages are kept, always including the page of the current (last) position.
+ *
+ * sd_quest_summarize writes the boxes of every logical page of every request (last_page_only = 0), or
+ * only of each request's last page (last_page_only != 0: after sd_append_kv added a row).
+ *   boxes   bf16 [num_pages][Hkv][2][d], device memory, 16-byte aligned, owned by the caller and kept
+ *           between calls: for physical page pg and KV head kvh, boxes[pg][kvh][0] is the minimum and
+ *           boxes[pg][kvh][1] the maximum over the page's positions < N_b (exact bf16 values).
+ *           Entries of pages no request holds are not written.
+ *   A page-table entry out of range is reported (SD_ERR_INDEX_OOB) and that page is skipped. */
+SD_API sd_status sd_quest_summarize(const sd_shape* shape, const void* K, const int32_t* page_table,
+                                    const int32_t* lens, void* boxes, int32_t last_page_only,
+                                    int32_t* dev_status, void* stream);
+
+/* sd_quest_index selects, per (b, h), ceil(k[b] / 16) pages: the current page (holding position
+ * N_b - 1) plus the most relevant others, relevance of page j being the largest q.k any key inside its
+ * box can reach, r_j = sum_d max(q_d * min_d, q_d * max_d) (fp32 accumulation of exact bf16 products);
+ * ties go to the lower page.  idx[b][h] receives every position < N_b of the kept pages, ascending,
+ * then -1 (the format sd_sparse_decode reads); when the budget covers every page, 0 .. N_b - 1.
+ *   boxes      as written by sd_quest_summarize for the current lengths.
+ *   k_max      must be at least 16 * ceil(k[b] / 16) for every b whose budget is below its page count,
+ *              and at least N_b where it is not (else SD_ERR_INVALID_ARG in dev_status, row all -1).
+ *   workspace  sd_workspace_size(shape, SD_OP_QUEST) bytes (the page relevance, fp32).
+ *   Supported up to 24576 pages per request (SD_ERR_UNSUPPORTED beyond). */
+SD_API sd_status sd_quest_index(const sd_shape* shape, const void* q, const void* boxes, const int32_t* page_table,
+                                const int32_t* lens, const int32_t* k, int32_t* idx, void* workspace,
+                                size_t workspace_bytes, int32_t* dev_status, void* stream);
 
 /* Static English text for a status code ("unknown status" for other values). */
 SD_API const char* sd_status_string(sd_status status);

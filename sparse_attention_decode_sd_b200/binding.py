@@ -27,9 +27,11 @@ SD_ERR_ORDER = 7
 SD_OP_TOPK = 1
 SD_OP_SPARSE = 2
 SD_OP_DENSE = 3
+SD_OP_QUEST = 4
 
 EXPORTED = ("sd_workspace_size", "sd_topk_index", "sd_topk_scores", "sd_topk_select", "sd_topk_index_static",
-            "sd_sparse_decode", "sd_dense_decode", "sd_append_kv", "sd_status_string", "sd_last_cuda_error", "sd_version")
+            "sd_sparse_decode", "sd_dense_decode", "sd_append_kv", "sd_quest_summarize", "sd_quest_index",
+            "sd_status_string", "sd_last_cuda_error", "sd_version")
 
 
 class SdShape(ctypes.Structure):
@@ -72,8 +74,10 @@ def load():
     lib.sd_sparse_decode.argtypes = [SH, P, P, P, P, P, P, P, P, SZ, P, P]
     lib.sd_dense_decode.argtypes = [SH, P, P, P, P, P, P, P, SZ, P, P]
     lib.sd_append_kv.argtypes = [SH, P, P, P, P, P, P, P, I32, P, P]
+    lib.sd_quest_summarize.argtypes = [SH, P, P, P, P, I32, P, P]
+    lib.sd_quest_index.argtypes = [SH, P, P, P, P, P, P, P, SZ, P, P]
     for f in (lib.sd_workspace_size, lib.sd_topk_index, lib.sd_topk_scores, lib.sd_topk_select, lib.sd_sparse_decode,
-              lib.sd_dense_decode, lib.sd_append_kv):
+              lib.sd_dense_decode, lib.sd_append_kv, lib.sd_quest_summarize, lib.sd_quest_index):
         f.restype = I32
     lib.sd_status_string.argtypes = [I32]
     lib.sd_status_string.restype = ctypes.c_char_p
@@ -179,6 +183,26 @@ def sd_dense_decode(shape, q, K, V, page_table, lens, out, workspace, dev_status
     st = load().sd_dense_decode(ctypes.byref(shape), _ptr(q), _ptr(K), _ptr(V), _ptr(page_table), _ptr(lens),
                                 _ptr(out), _ptr(workspace), _ws_bytes(workspace), _ptr(dev_status), _stream(stream))
     return _check(st, "sd_dense_decode", check)
+
+
+def sd_quest_summarize(shape, K, page_table, lens, boxes, dev_status, last_page_only=False, stream=None,
+                       check=True) -> int:
+    st = load().sd_quest_summarize(ctypes.byref(shape), _ptr(K), _ptr(page_table), _ptr(lens), _ptr(boxes),
+                                   int(bool(last_page_only)), _ptr(dev_status), _stream(stream))
+    return _check(st, "sd_quest_summarize", check)
+
+
+def sd_quest_index(shape, q, boxes, page_table, lens, k, idx, workspace, dev_status, stream=None, check=True) -> int:
+    st = load().sd_quest_index(ctypes.byref(shape), _ptr(q), _ptr(boxes), _ptr(page_table), _ptr(lens), _ptr(k),
+                               _ptr(idx), _ptr(workspace), ctypes.c_size_t(workspace.numel()), _ptr(dev_status),
+                               _stream(stream))
+    return _check(st, "sd_quest_index", check)
+
+
+def quest_boxes_for(shape: SdShape, device=None) -> torch.Tensor:
+    """A caller-side buffer for the Quest page boxes: bf16 [num_pages][Hkv][2][head_dim]."""
+    return torch.empty((shape.num_pages, shape.num_kv_heads, 2, shape.head_dim), dtype=torch.bfloat16,
+                       device=device or "cuda")
 
 
 def sd_append_kv(shape, K, V, page_table, lens, k_new, v_new, k_sel, ratio, dev_status, stream=None,

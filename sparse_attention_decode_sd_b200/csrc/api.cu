@@ -202,6 +202,7 @@ sd_status sd_workspace_size(const sd_shape* shape, int32_t op, size_t* bytes) {
         case SD_OP_TOPK: *bytes = topk_workspace(d); return SD_OK;
         case SD_OP_SPARSE:
         case SD_OP_DENSE: *bytes = decode_workspace(d); return SD_OK;
+        case SD_OP_QUEST: *bytes = align256((size_t)d.B * d.Hq * d.max_pages * sizeof(float)); return SD_OK;
         default: return SD_ERR_INVALID_ARG;
     }
 }
@@ -348,6 +349,74 @@ sd_status sd_append_kv(const sd_shape* shape, void* K, void* V, const int32_t* p
     a.num_pages = d.num_pages;
     a.ratio = ratio;
     return launch_status(launch_append(a, static_cast<cudaStream_t>(stream)));
+}
+
+namespace {
+
+sd_status quest_args(const sd_shape* shape, QuestArgs* a, Dims* d) {
+    sd_status st = check_shape(shape, d);
+    if (st != SD_OK) return st;
+    *a = QuestArgs{};
+    a->B = d->B;
+    a->Hq = d->Hq;
+    a->Hkv = d->Hkv;
+    a->G = d->G;
+    a->max_pages = d->max_pages;
+    a->num_pages = d->num_pages;
+    a->k_max = d->k_max;
+    a->n_cap = d->n_cap;
+    return SD_OK;
+}
+
+}  // namespace
+
+sd_status sd_quest_summarize(const sd_shape* shape, const void* K, const int32_t* page_table, const int32_t* lens,
+                             void* boxes, int32_t last_page_only, int32_t* dev_status, void* stream) {
+    QuestArgs a;
+    Dims d;
+    sd_status st = quest_args(shape, &a, &d);
+    if (st != SD_OK) return st;
+    if (!K || !page_table || !lens || !boxes || !dev_status) return SD_ERR_INVALID_ARG;
+    if (!aligned(K, 16) || !aligned(boxes, 16) || !aligned(page_table, 4) || !aligned(lens, 4) ||
+        !aligned(dev_status, 4))
+        return SD_ERR_INVALID_ARG;
+    if (!last_page_only && (long)d.B * d.max_pages * d.Hkv >= (1L << 36)) return SD_ERR_UNSUPPORTED;
+    a.K = static_cast<const __nv_bfloat16*>(K);
+    a.boxes = static_cast<__nv_bfloat16*>(boxes);
+    a.page_table = page_table;
+    a.lens = lens;
+    a.status = dev_status;
+    a.last_only = last_page_only ? 1 : 0;
+    return launch_status(launch_quest_summarize(a, static_cast<cudaStream_t>(stream)));
+}
+
+sd_status sd_quest_index(const sd_shape* shape, const void* q, const void* boxes, const int32_t* page_table,
+                         const int32_t* lens, const int32_t* k, int32_t* idx, void* workspace, size_t workspace_bytes,
+                         int32_t* dev_status, void* stream) {
+    QuestArgs a;
+    Dims d;
+    sd_status st = quest_args(shape, &a, &d);
+    if (st != SD_OK) return st;
+    if (!q || !boxes || !page_table || !lens || !k || !idx || !workspace || !dev_status) return SD_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(boxes, 16) || !aligned(page_table, 4) || !aligned(lens, 4) || !aligned(k, 4) ||
+        !aligned(idx, 4) || !aligned(workspace, 256) || !aligned(dev_status, 4))
+        return SD_ERR_INVALID_ARG;
+    if (d.max_pages > kQuestMaxPages) return SD_ERR_UNSUPPORTED;
+    size_t need = 0;
+    sd_workspace_size(shape, SD_OP_QUEST, &need);
+    if (workspace_bytes < need) return SD_ERR_WORKSPACE;
+    a.q = static_cast<const __nv_bfloat16*>(q);
+    a.boxes = const_cast<__nv_bfloat16*>(static_cast<const __nv_bfloat16*>(boxes));
+    a.page_table = page_table;
+    a.lens = lens;
+    a.k = k;
+    a.idx = idx;
+    a.rel = static_cast<float*>(workspace);
+    a.status = dev_status;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    st = launch_status(launch_quest_score(a, s));
+    if (st != SD_OK) return st;
+    return launch_status(launch_quest_select(a, s));
 }
 
 const char* sd_status_string(sd_status status) {

@@ -81,6 +81,28 @@ cudaError_t launch_union(const DecodeArgs& a, bool dense, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs& a, bool dense, cudaStream_t stream);
 cudaError_t launch_merge(const DecodeArgs& a, cudaStream_t stream);
 
+// Quest page-level indexer.
+constexpr int kQuestMaxPages = 24 * 1024;   // pages per request the page select holds in shared memory
+
+struct QuestArgs {
+    const __nv_bfloat16* q;
+    const __nv_bfloat16* K;
+    __nv_bfloat16* boxes;        // [num_pages][Hkv][2][128]: per-dimension minimum, then maximum
+    const int32_t* page_table;
+    const int32_t* lens;
+    const int32_t* k;
+    int32_t* idx;
+    float* rel;                  // workspace [B][Hq][max_pages]: page relevance
+    int32_t* status;
+    int B, Hq, Hkv, G, max_pages, num_pages, k_max;
+    long n_cap;
+    int last_only;               // summarize: only each request's last page
+};
+cudaError_t launch_quest_summarize(const QuestArgs& a, cudaStream_t stream);
+cudaError_t launch_quest_score(const QuestArgs& a, cudaStream_t stream);
+cudaError_t launch_quest_select(const QuestArgs& a, cudaStream_t stream);
+size_t quest_select_smem(const QuestArgs& a);
+
 struct AppendArgs {
     __nv_bfloat16* K;
     __nv_bfloat16* V;
