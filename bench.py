@@ -449,6 +449,135 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def run_study(args):
+    """Indexer-inclusive end-to-end study: for each sparsity ratio of the sweep workload, the step time of
+    exact index + decode and of Quest index + decode, against dense decode at the same shape.  Each
+    point runs in its own process (this script, single GPU)."""
+    import subprocess
+    points = []
+    for ratio in wl.SWEEP_RATIOS:
+        for indexer in ("exact", "quest"):
+            cmd = [sys.executable, os.path.abspath(__file__), "--workload", "sweep128k", "--ratio", str(ratio),
+                   "--indexer", indexer, "--steps", str(args.steps), "--warmup", str(args.warmup),
+                   "--no-cpu-baseline"] + (["--no-dense"] if indexer == "quest" else [])
+            r = subprocess.run(cmd, capture_output=True, text=True, check=True)
+            line = json.loads(r.stdout.strip().splitlines()[-1])
+            point = {"ratio": ratio, "indexer": indexer, "ms_per_step": line["ms_per_step"],
+                     "tokens_per_s": line["value"], "kernels": {k: v["ms"] for k, v in line["kernels"].items()}}
+            if indexer == "exact":
+                point["dense_decode_ms"] = line["kernels"].get("dense_decode", {}).get("ms")
+            points.append(point)
+            print(json.dumps(point), flush=True)
+    dense = {p["ratio"]: p["dense_decode_ms"] for p in points if p["indexer"] == "exact"}
+    summary = {"study": "index + decode vs dense decode, sweep128k (B=16, 32/8 heads, N=131072)",
+               "speedup_vs_dense": {f"{p['indexer']}@N/{p['ratio']}": dense[p["ratio"]] / p["ms_per_step"]
+                                    for p in points if dense.get(p["ratio"])}}
+    print(json.dumps(summary), flush=True)
+
+
+def quest_k_max(w) -> int:
+    """Row length that holds every Quest selection of w (whole pages, or the whole context)."""
+    need = 1
+    for n, k in zip(w.lens.tolist(), w.k.tolist()):
+        np_ = (n + w.P - 1) // w.P
+        kp = min(np_, (k + w.P - 1) // w.P)
+        need = max(need, n if kp >= np_ else kp * w.P)
+    return need
+
+
+def run_quest(args):
+    """The step with the Quest page-level indexer in place of the exact one: refresh each request's
+    last page box (what a decode loop does after appending), select pages, sparse decode."""
+    world, rank, local = dist_setup()
+    dev = torch.device("cuda", local)
+    kw = {"ratio": args.ratio} if args.workload == "sweep128k" else {}
+    w = wl.named(args.workload, device=dev, seed=rank_seed(args.workload, rank), **kw)
+    k_max = quest_k_max(w)
+    shape = sdb.make_shape(w.B, w.Hq, w.Hkv, w.max_pages, k_max, w.num_pages)
+    boxes = sdb.quest_boxes_for(shape, dev)
+    ws_q = sdb.workspace_for(shape, sdb.SD_OP_QUEST, dev)
+    ws_dec = sdb.workspace_for(shape, sdb.SD_OP_SPARSE, dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    idx = torch.full((w.B, w.Hq, k_max), -1, dtype=torch.int32, device=dev)
+    out = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device=dev)
+    flush = torch.zeros(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sdb.sd_quest_summarize(shape, w.K, w.page_table, w.lens, boxes, status, stream=stream)   # the prefill's part
+
+    def index():
+        sdb.sd_quest_summarize(shape, w.K, w.page_table, w.lens, boxes, status, last_page_only=True, stream=stream)
+        sdb.sd_quest_index(shape, w.q, boxes, w.page_table, w.lens, w.k, idx, ws_q, status, stream)
+
+    for _ in range(args.warmup):
+        flush.amax()
+        index()
+        sdb.sd_sparse_decode(shape, w.q, w.K, w.V, w.page_table, w.lens, idx, out, ws_dec, status, stream)
+    torch.cuda.synchronize()
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())}: {sdb.status_string(int(status.item()))}")
+    sampler = ClockSampler(local)
+    sampler.start()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.amax()
+        e = ev[i]
+        e[0].record(stream)
+        index()
+        e[1].record(stream)
+        sdb.sd_sparse_decode(shape, w.q, w.K, w.V, w.page_table, w.lens, idx, out, ws_dec, status, stream)
+        e[2].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop()
+    t_index = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
+    t_decode = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
+    t_step_max = max_over_ranks(world, sum(e[0].elapsed_time(e[2]) for e in ev) / args.steps)
+    if rank != 0:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+    hbm, peak_kind = peaks()
+    lens = w.lens.long()
+    pages = int(((lens + w.P - 1) // w.P).sum())
+    q_bytes, out_bytes = w.B * w.Hq * w.d * 2, w.B * w.Hq * w.d * 4
+    idx_bytes = int((idx >= 0).sum()) * 4
+    U = union_rows(w, idx)
+    # Eq. 10's page representation: min and max rows (2 x d bf16) per page and KV head, plus q
+    index_bytes = pages * w.Hkv * 2 * w.d * 2 + q_bytes
+    decode_bytes = U * 2 * w.d * 2 + q_bytes + idx_bytes + out_bytes
+
+    def gbs(nbytes, ms):
+        return nbytes / (ms / 1e3) / 1e9
+
+    kernels = {"quest_index": {"ms": t_index, "bytes": index_bytes, "gbs": gbs(index_bytes, t_index),
+                               "frac": gbs(index_bytes, t_index) / hbm},
+               "sparse_decode": {"ms": t_decode, "bytes": decode_bytes, "gbs": gbs(decode_bytes, t_decode),
+                                 "frac": gbs(decode_bytes, t_decode) / hbm}}
+    cfg = config_of(w, args, world)
+    cfg["indexer"] = "quest (page boxes, ceil(k/16) pages incl. the current one)"
+    line = {
+        "metric": METRIC, "value": job_tokens_per_s(world, w.B, t_step_max), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_step_max, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded bf16 N(0,1) q/K/V, structure per workload)", "config": cfg,
+        "required_bytes_per_step": index_bytes + decode_bytes, "union_rows": U,
+        "effective_hbm_gbs": gbs(index_bytes + decode_bytes, t_step_max),
+        "effective_hbm_frac": gbs(index_bytes + decode_bytes, t_step_max) / hbm,
+        "kernels": kernels,
+        "roofline": {"bound": "hbm", "kernel": "decode_kernel", "achieved": kernels["sparse_decode"]["gbs"],
+                     "peak": hbm, "unit": "GB/s", "frac": kernels["sparse_decode"]["frac"], "peak_source": peak_kind,
+                     "traffic": None, "algorithmic_bytes": decode_bytes},
+        "clocks": clocks, "gpu_launches": 7 * args.steps,
+    }
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -457,13 +586,22 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="long128k", choices=sorted(wl.CONFIG_IDS))
     ap.add_argument("--ratio", type=int, default=50, help="sparsity ratio of the sweep128k workload")
+    ap.add_argument("--indexer", choices=("exact", "quest"), default="exact",
+                    help="exact top-k (the method) or the Quest page-level approximate indexer")
+    ap.add_argument("--study", action="store_true",
+                    help="index + decode against dense decode over the sparsity sweep (sweep128k: N/10, N/50, "
+                         "N/100, N), exact and Quest indexers; one JSON line per point, then a summary line")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    if args.impl == "reference":
+    if args.study:
+        run_study(args)
+    elif args.impl == "reference":
         run_reference(args)
+    elif args.indexer == "quest":
+        run_quest(args)
     else:
         run_ours(args)
 
