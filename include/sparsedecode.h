@@ -192,6 +192,13 @@ SD_API sd_status sd_quest_index(const sd_shape* shape, const void* q, const void
                                 const int32_t* lens, const int32_t* k, int32_t* idx, void* workspace,
                                 size_t workspace_bytes, int32_t* dev_status, void* stream);
 
+/* Self-test of failure detection (no counterpart in the pages): launches one warp that waits, with
+ * the bounded-wait helper every pipeline wait of the library uses, on a barrier that nothing completes.
+ * The wait gives up after wait_ms (1 .. 10000) and stores SD_ERR_TIMEOUT in dev_status; the kernel
+ * issues no copy, so it leaves nothing in flight and the context stays usable.  Asynchronous on stream;
+ * read dev_status after synchronising. */
+SD_API sd_status sd_selftest_wait_timeout(uint32_t wait_ms, int32_t* dev_status, void* stream);
+
 /* Static English text for a status code ("unknown status" for other values). */
 SD_API const char* sd_status_string(sd_status status);
 

@@ -31,7 +31,7 @@ SD_OP_QUEST = 4
 
 EXPORTED = ("sd_workspace_size", "sd_topk_index", "sd_topk_scores", "sd_topk_select", "sd_topk_index_static",
             "sd_sparse_decode", "sd_dense_decode", "sd_append_kv", "sd_quest_summarize", "sd_quest_index",
-            "sd_status_string", "sd_last_cuda_error", "sd_version")
+            "sd_selftest_wait_timeout", "sd_status_string", "sd_last_cuda_error", "sd_version")
 
 
 class SdShape(ctypes.Structure):
@@ -76,6 +76,8 @@ def load():
     lib.sd_append_kv.argtypes = [SH, P, P, P, P, P, P, P, I32, P, P]
     lib.sd_quest_summarize.argtypes = [SH, P, P, P, P, I32, P, P]
     lib.sd_quest_index.argtypes = [SH, P, P, P, P, P, P, P, SZ, P, P]
+    lib.sd_selftest_wait_timeout.argtypes = [ctypes.c_uint32, P, P]
+    lib.sd_selftest_wait_timeout.restype = I32
     for f in (lib.sd_workspace_size, lib.sd_topk_index, lib.sd_topk_scores, lib.sd_topk_select, lib.sd_sparse_decode,
               lib.sd_dense_decode, lib.sd_append_kv, lib.sd_quest_summarize, lib.sd_quest_index):
         f.restype = I32
@@ -197,6 +199,11 @@ def sd_quest_index(shape, q, boxes, page_table, lens, k, idx, workspace, dev_sta
                                _ptr(idx), _ptr(workspace), ctypes.c_size_t(workspace.numel()), _ptr(dev_status),
                                _stream(stream))
     return _check(st, "sd_quest_index", check)
+
+
+def sd_selftest_wait_timeout(wait_ms: int, dev_status, stream=None, check=True) -> int:
+    st = load().sd_selftest_wait_timeout(int(wait_ms), _ptr(dev_status), _stream(stream))
+    return _check(st, "sd_selftest_wait_timeout", check)
 
 
 def quest_boxes_for(shape: SdShape, device=None) -> torch.Tensor:

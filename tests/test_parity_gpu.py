@@ -302,3 +302,19 @@ def test_bad_k_and_length_are_reported():
     w.lens[1] = w.max_pages * w.P + 1
     r.dense()
     assert r.device_status() == sdb.SD_ERR_INVALID_ARG
+
+
+def test_bounded_wait_gives_up_and_the_context_survives():
+    """Failure detection without a fault: a device-side wait on a barrier nothing completes gives up after
+    its limit and records SD_ERR_TIMEOUT; the context then still runs the indexer and decode correctly."""
+    import time
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    sdb.sd_selftest_wait_timeout(50, st)
+    torch.cuda.synchronize()
+    dt = time.perf_counter() - t0
+    assert int(st.item()) == sdb.SD_ERR_TIMEOUT
+    assert 0.045 <= dt < 5.0, dt
+    w_cpu = wl.make_workload(1, 8, 2, 3000, 50, seed=91)
+    _run_small(w_cpu)
