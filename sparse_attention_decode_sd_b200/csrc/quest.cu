@@ -43,11 +43,16 @@ __global__ void __launch_bounds__(256) quest_summarize_kernel(QuestArgs a, long 
         return;
     }
     const int rows = min(kPageSize, n - j * kPageSize);
+    // all 16 row loads in flight together (rows past N_b repeat row 0, which leaves min and max unchanged)
+    uint2 v[kPageSize];
+#pragma unroll
+    for (int r = 0; r < kPageSize; ++r)
+        v[r] = *reinterpret_cast<const uint2*>(a.K + (((long)page * kPageSize + (r < rows ? r : 0)) * a.Hkv + kvh) *
+                                                   kHeadDim + 4 * lane);
     float mn[4], mx[4];
-    for (int r = 0; r < rows; ++r) {
-        const uint2 v = *reinterpret_cast<const uint2*>(a.K + (((long)page * kPageSize + r) * a.Hkv + kvh) * kHeadDim +
-                                                        4 * lane);
-        const float f[4] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y)};
+#pragma unroll
+    for (int r = 0; r < kPageSize; ++r) {
+        const float f[4] = {bf16_lo(v[r].x), bf16_hi(v[r].x), bf16_lo(v[r].y), bf16_hi(v[r].y)};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             mn[e] = r ? fminf(mn[e], f[e]) : f[e];

@@ -52,6 +52,10 @@ __device__ __forceinline__ void select_bin(const int* hist, int nbins, int targe
 // greater than T.  The keys' range is found first and the digits (up to 12 bits each) start at the
 // highest bit in which the smallest and largest key differ: candidates cluster just above a
 // threshold, so a fixed top digit would pile them into a few contended histogram bins.
+// When the bin holding the target after a digit has at most kSmallBin elements, they are collected and
+// ranked directly by one warp instead of running the next digit's histogram.
+constexpr int kSmallBin = 64;
+
 template <class Visit>
 __device__ void radix_select(Visit visit, int target, int* hist, int* scratch, int* s_sel, uint32_t* T_out,
                              int* greater_out) {
@@ -95,10 +99,55 @@ __device__ void radix_select(Visit visit, int target, int* hist, int* scratch, i
         });
         __syncthreads();
         select_bin(hist, nb, target - greater, scratch, s_sel);
-        prefix |= (uint32_t)s_sel[0] << sh;
+        const int bin = s_sel[0];
+        const int in_bin = hist[bin];
+        prefix |= (uint32_t)bin << sh;
         greater += s_sel[1];
         top = sh - 1;
         __syncthreads();
+        if (top >= 0 && in_bin <= kSmallBin) {
+            // the few keys of the bin (their bits above `top` equal prefix's): collect and rank them
+            uint32_t* list = reinterpret_cast<uint32_t*>(hist);   // [kSmallBin]
+            int* count = hist + kSmallBin;
+            if (tid == 0) *count = 0;
+            __syncthreads();
+            visit([&](uint32_t key) {
+                if ((key >> (top + 1)) == (prefix >> (top + 1))) list[atomicAdd(count, 1)] = key;
+            });
+            __syncthreads();
+            if (tid < 32) {
+                const int m = *count, r = target - greater;   // r-th largest of the m keys, 1 <= r <= m
+                uint32_t found = 0u;
+                int above = 0;
+                bool hit = false;
+                for (int i = lane; i < m; i += 32) {
+                    const uint32_t e = list[i];
+                    int gt = 0, eq = 0;
+                    for (int t = 0; t < m; ++t) {
+                        gt += list[t] > e;
+                        eq += list[t] == e;
+                    }
+                    if (gt < r && r <= gt + eq) {
+                        found = e;
+                        above = gt;
+                        hit = true;
+                    }
+                }
+                const uint32_t who = __ballot_sync(0xffffffffu, hit);
+                const int src = who ? __ffs(who) - 1 : 0;
+                found = __shfl_sync(0xffffffffu, found, src);
+                above = __shfl_sync(0xffffffffu, above, src);
+                if (lane == 0) {
+                    s_sel[0] = (int)found;
+                    s_sel[1] = above;
+                }
+            }
+            __syncthreads();
+            prefix = (uint32_t)s_sel[0];
+            greater += s_sel[1];
+            __syncthreads();
+            break;
+        }
     }
     *T_out = prefix;       // all keys equal: T is that key, none greater
     *greater_out = greater;
