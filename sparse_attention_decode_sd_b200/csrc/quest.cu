@@ -107,25 +107,12 @@ __device__ __forceinline__ void load_q_signed(const QuestArgs& a, int b, int kvh
     }
 }
 
-template <int NT>
-__global__ void __launch_bounds__(256) quest_score_kernel(QuestArgs a, long units) {
-    pdl_enter();
+constexpr int kQuestTilesPerWarp = 8;   // 16-page tiles a warp scores, with the next tile's loads in flight
+
+// Box fragments of tile j0 (pages j0 + g and j0 + g + 8; pages past the request read page 0's box).
+__device__ __forceinline__ void load_box_tile(const QuestArgs& a, int b, int kvh, int np, int j0, uint32_t (&Rmx)[2][16],
+                                              uint32_t (&Rmn)[2][16]) {
     const int lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
-    const long u = (long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    if (u >= units) return;
-    const int tiles = (a.max_pages + 15) / 16;
-    const int tile = (int)(u % tiles);
-    const long grp = u / tiles;
-    const int b = (int)(grp / a.Hkv), kvh = (int)(grp % a.Hkv);
-    const int n = checked_len(a.lens, b, a.n_cap, a.status);
-    const int np = (n + kPageSize - 1) / kPageSize;
-    const int j0 = tile * 16;
-    if (j0 >= np) return;
-    uint32_t qp[NT][16], qn[NT][16];
-    load_q_signed<NT>(a, b, kvh, false, qp);
-    load_q_signed<NT>(a, b, kvh, true, qn);
-    // A operand rows: pages j0 + g and j0 + g + 8 (pages past the request read page 0's box, unused)
-    uint32_t Rmx[2][16], Rmn[2][16];
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
         const int j = j0 + g + 8 * half;
@@ -135,28 +122,54 @@ __global__ void __launch_bounds__(256) quest_score_kernel(QuestArgs a, long unit
         load_row_frags(box + kHeadDim, c, Rmx[half]);
         load_row_frags(box, c, Rmn[half]);
     }
-    float acc[NT][4];
+}
+
+// One warp per (request, kv head, kQuestTilesPerWarp consecutive 16-page tiles).
+template <int NT>
+__global__ void __launch_bounds__(256) quest_score_kernel(QuestArgs a, long units) {
+    pdl_enter();
+    const int lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
+    const long u = (long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (u >= units) return;
+    const int chunks = (a.max_pages + 16 * kQuestTilesPerWarp - 1) / (16 * kQuestTilesPerWarp);
+    const int chunk = (int)(u % chunks);
+    const long grp = u / chunks;
+    const int b = (int)(grp / a.Hkv), kvh = (int)(grp % a.Hkv);
+    const int n = checked_len(a.lens, b, a.n_cap, a.status);
+    const int np = (n + kPageSize - 1) / kPageSize;
+    const int jbeg = chunk * 16 * kQuestTilesPerWarp, jend = min(np, jbeg + 16 * kQuestTilesPerWarp);
+    if (jbeg >= jend) return;
+    uint32_t qp[NT][16], qn[NT][16];
+    load_q_signed<NT>(a, b, kvh, false, qp);
+    load_q_signed<NT>(a, b, kvh, true, qn);
+    uint32_t Rmx[2][16], Rmn[2][16];
+    load_box_tile(a, b, kvh, np, jbeg, Rmx, Rmn);
+    for (int j0 = jbeg; j0 < jend; j0 += 16) {
+        float acc[NT][4];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+        for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
 #pragma unroll
-    for (int s = 0; s < 8; ++s)
+        for (int s = 0; s < 8; ++s)
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            mma_bf16_16816(acc[nt], Rmx[0][2 * s], Rmx[1][2 * s], Rmx[0][2 * s + 1], Rmx[1][2 * s + 1], qp[nt][2 * s],
-                           qp[nt][2 * s + 1]);
-            mma_bf16_16816(acc[nt], Rmn[0][2 * s], Rmn[1][2 * s], Rmn[0][2 * s + 1], Rmn[1][2 * s + 1], qn[nt][2 * s],
-                           qn[nt][2 * s + 1]);
-        }
+            for (int nt = 0; nt < NT; ++nt) {
+                mma_bf16_16816(acc[nt], Rmx[0][2 * s], Rmx[1][2 * s], Rmx[0][2 * s + 1], Rmx[1][2 * s + 1],
+                               qp[nt][2 * s], qp[nt][2 * s + 1]);
+                mma_bf16_16816(acc[nt], Rmn[0][2 * s], Rmn[1][2 * s], Rmn[0][2 * s + 1], Rmn[1][2 * s + 1],
+                               qn[nt][2 * s], qn[nt][2 * s + 1]);
+            }
+        // the next tile's loads go out before this tile's results are written
+        if (j0 + 16 < jend) load_box_tile(a, b, kvh, np, j0 + 16, Rmx, Rmn);
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const int col = nt * 8 + 2 * c + e;
-            if (col >= a.G) continue;
-            float* rrow = a.rel + ((long)b * a.Hq + (long)kvh * a.G + col) * a.max_pages;
-            if (j0 + g < np) rrow[j0 + g] = acc[nt][e];
-            if (j0 + g + 8 < np) rrow[j0 + g + 8] = acc[nt][2 + e];
-        }
+            for (int e = 0; e < 2; ++e) {
+                const int col = nt * 8 + 2 * c + e;
+                if (col >= a.G) continue;
+                float* rrow = a.rel + ((long)b * a.Hq + (long)kvh * a.G + col) * a.max_pages;
+                if (j0 + g < np) rrow[j0 + g] = acc[nt][e];
+                if (j0 + g + 8 < np) rrow[j0 + g + 8] = acc[nt][2 + e];
+            }
+    }
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -237,7 +250,7 @@ cudaError_t launch_quest_summarize(const QuestArgs& a, cudaStream_t stream) {
 }
 
 cudaError_t launch_quest_score(const QuestArgs& a, cudaStream_t stream) {
-    const long units = (long)a.B * a.Hkv * ((a.max_pages + 15) / 16);
+    const long units = (long)a.B * a.Hkv * ((a.max_pages + 16 * kQuestTilesPerWarp - 1) / (16 * kQuestTilesPerWarp));
     const long grid = (units + 7) / 8;
     cudaError_t e = a.G <= 8 ? launch_pdl(quest_score_kernel<1>, dim3((unsigned)grid), dim3(256), 0, stream, a, units)
                              : launch_pdl(quest_score_kernel<2>, dim3((unsigned)grid), dim3(256), 0, stream, a, units);
