@@ -37,8 +37,10 @@ from sparse_attention_decode_sd_b200 import workloads as wl  # noqa: E402
 
 METRIC = "decode tokens/s and effective HBM GB/s (% of roofline) at 128K ctx, 50x sparsity"
 L2_FLUSH_BYTES = 512 << 20
-# kernels of one step: threshold, score pass, select; prep, union, decode, merge
-LAUNCHES_PER_STEP = 7
+# kernels of one step: threshold, score pass, select; rows, sparse decode
+LAUNCHES_PER_STEP = 5
+# kernels of one Quest step: last-page box refresh, page score, page select; rows, sparse decode
+QUEST_LAUNCHES_PER_STEP = 5
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -63,7 +65,7 @@ def source_hash(*names):
 KERNEL_SOURCES = {
     "score_pass_kernel": ("topk_score.cu", "common.cuh", "kernels.h"),
     "select_kernel": ("topk_select.cu", "common.cuh", "kernels.h"),
-    "decode_kernel": ("sparse_decode.cu", "common.cuh", "kernels.h"),
+    "sparse_decode_kernel": ("sparse_decode.cu", "common.cuh", "kernels.h"),
 }
 
 
@@ -358,14 +360,15 @@ def run_ours(args):
     dense_ms = None
     if not args.no_dense:
         dout = torch.empty_like(out)
+        ws_dense = sdb.workspace_for(shape, sdb.SD_OP_DENSE, dev)
         dev_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(5)]
         for _ in range(2):
             flush_l2()
-            sdb.sd_dense_decode(shape, w.q, w.K, w.V, w.page_table, w.lens, dout, ws_dec, status, stream)
+            sdb.sd_dense_decode(shape, w.q, w.K, w.V, w.page_table, w.lens, dout, ws_dense, status, stream)
         for a, b_ in dev_ev:
             flush_l2()
             a.record(stream)
-            sdb.sd_dense_decode(shape, w.q, w.K, w.V, w.page_table, w.lens, dout, ws_dec, status, stream)
+            sdb.sd_dense_decode(shape, w.q, w.K, w.V, w.page_table, w.lens, dout, ws_dense, status, stream)
             b_.record(stream)
         torch.cuda.synchronize()
         dense_ms = statistics.mean(a.elapsed_time(b_) for a, b_ in dev_ev)
@@ -420,7 +423,7 @@ def run_ours(args):
                                    "frac": gbs(req["dense_decode"], dense_ms) / hbm}
     # dominant kernel of the step by time
     dom = "topk_scores" if t_scores >= t_decode else "sparse_decode"
-    dom_kernel = {"topk_scores": "score_pass_kernel", "sparse_decode": "decode_kernel"}[dom]
+    dom_kernel = {"topk_scores": "score_pass_kernel", "sparse_decode": "sparse_decode_kernel"}[dom]
     roofline = {"bound": "hbm", "kernel": dom_kernel, "achieved": kernels[dom]["gbs"], "peak": hbm, "unit": "GB/s",
                 "frac": kernels[dom]["gbs"] / hbm, "peak_source": peak_kind,
                 "traffic": traffic_from_profiles(dom_kernel, w.name),
@@ -567,10 +570,10 @@ def run_quest(args):
         "effective_hbm_gbs": gbs(index_bytes + decode_bytes, t_step_max),
         "effective_hbm_frac": gbs(index_bytes + decode_bytes, t_step_max) / hbm,
         "kernels": kernels,
-        "roofline": {"bound": "hbm", "kernel": "decode_kernel", "achieved": kernels["sparse_decode"]["gbs"],
+        "roofline": {"bound": "hbm", "kernel": "sparse_decode_kernel", "achieved": kernels["sparse_decode"]["gbs"],
                      "peak": hbm, "unit": "GB/s", "frac": kernels["sparse_decode"]["frac"], "peak_source": peak_kind,
                      "traffic": None, "algorithmic_bytes": decode_bytes},
-        "clocks": clocks, "gpu_launches": 7 * args.steps,
+        "clocks": clocks, "gpu_launches": QUEST_LAUNCHES_PER_STEP * args.steps,
     }
     print(json.dumps(line), flush=True)
     if world > 1:

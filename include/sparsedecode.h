@@ -24,7 +24,8 @@
  *               are never read.
  *   lens        int32 [B], device memory: context length N_b, 0 <= N_b <= max_pages_per_req * P.
  *   idx         int32 [B][Hq][k_max], device memory: per (b, h) the selected positions in strictly
- *               ascending order, followed by -1 padding.  Any negative entry counts as padding.
+ *               ascending order, followed by padding (any negative value, -1 by convention).  A
+ *               non-negative entry after padding is an ordering error (SD_ERR_ORDER).
  *   out         fp32 [B][Hq][d], device memory, 16-byte aligned.
  *   workspace   device scratch owned by the caller, at least sd_workspace_size() bytes,
  *               256-byte aligned.  Its contents need no initialisation and are not preserved.
@@ -138,10 +139,12 @@ SD_API sd_status sd_topk_index_static(const sd_shape* shape, const void* q, cons
 /* Sparse decode attention over the selected rows ("Sparse" mode of Fig. 1(a) of "Inference-time
  * context sparsity"; SDPA of the xllm survey sec. 1.1 restricted to the selected set).
  *   out[b,h] = sum_{i in S} w_i V[b, h/G, i],  w = softmax over S of (q[b,h] . K[b,h/G,i]) / sqrt(d),
- *   S = the non-negative entries of idx[b][h].  An empty S gives out = 0.
- *   Each GQA group reads the union of its heads' selected rows once.
- *   Device checks: entries must be < N_b (SD_ERR_INDEX_OOB) and strictly ascending
- *   (SD_ERR_ORDER). */
+ *   S = the entries of idx[b][h] before its first negative one.  An empty S gives out = 0.
+ *   Each query head gathers its own rows; the heads of a GQA group are processed side by side, so a
+ *   row that several of them selected is read from HBM about once and from L2 after that.
+ *   Device checks: entries must be < N_b and map to a page-table entry in range (SD_ERR_INDEX_OOB),
+ *   strictly ascending, with nothing but padding after the first negative entry (SD_ERR_ORDER).
+ *   B * Hq * k_max must be below 2^31 (else SD_ERR_UNSUPPORTED, also from sd_workspace_size). */
 SD_API sd_status sd_sparse_decode(const sd_shape* shape, const void* q, const void* K, const void* V,
                            const int32_t* page_table, const int32_t* lens, const int32_t* idx, float* out,
                            void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream);

@@ -50,9 +50,9 @@ sd_status device_info(DeviceInfo* out) {
 struct Dims {
     int B, Hq, Hkv, G, max_pages, k_max, num_pages;
     long n_cap;   // max_pages * page size
-    int nr;       // union-building ranges per (b, kv head) group
+    int nr;       // dense decode: counted ranges per (b, kv head) group
     int nrt;      // B * Hkv * nr
-    int jmax;     // decode segment slots per (b, h)
+    int jmax;     // dense decode: segment slots per (b, h)
 };
 
 sd_status check_shape(const sd_shape* s, Dims* d) {
@@ -69,7 +69,7 @@ sd_status check_shape(const sd_shape* s, Dims* d) {
     if ((long)s->num_pages * kPageSize * s->num_kv_heads >= (1L << 32)) return SD_ERR_UNSUPPORTED;   // row index is 32-bit
     const long nr = (n_cap + kRange - 1) / kRange;
     const long nrt = (long)s->batch * s->num_kv_heads * nr;
-    if (nrt * kRange >= (1L << 31)) return SD_ERR_UNSUPPORTED;   // union rows are counted in int32
+    if (nrt * kRange >= (1L << 31)) return SD_ERR_UNSUPPORTED;   // rows are counted in int32
     d->B = s->batch;
     d->Hq = s->num_q_heads;
     d->Hkv = s->num_kv_heads;
@@ -104,23 +104,53 @@ TopkLayout topk_layout(const Dims& d) {
 }
 size_t topk_workspace(const Dims& d) { return topk_layout(d).total; }
 
-// decode workspace, in order: acc [B][Hq][jmax][128] fp32, ml [B][Hq][jmax] float2,
-// entries [nrt][kRange] uint2, counts [nrt], hdr [4] followed by per-group totals [B * Hkv]
-struct DecodeLayout {
-    size_t acc, ml, entries, counts, hdr, total;
+// dense decode workspace, in order: acc [B][Hq][jmax][128] fp32, ml [B][Hq][jmax] float2, counts [nrt],
+// hdr [4] followed by per-group totals [B * Hkv]
+struct DenseLayout {
+    size_t acc, ml, counts, hdr, total;
 };
-DecodeLayout decode_layout(const Dims& d) {
-    DecodeLayout L;
+DenseLayout dense_layout(const Dims& d) {
+    DenseLayout L;
     const size_t slots = (size_t)d.B * d.Hq * d.jmax;
     L.acc = 0;
     L.ml = L.acc + align256(slots * kHeadDim * sizeof(float));
-    L.entries = L.ml + align256(slots * sizeof(float2));
-    L.counts = L.entries + align256((size_t)d.nrt * kRange * sizeof(uint2));
+    L.counts = L.ml + align256(slots * sizeof(float2));
     L.hdr = L.counts + align256((size_t)d.nrt * sizeof(int));
     L.total = L.hdr + align256((4 + (size_t)d.B * d.Hkv) * sizeof(int));
     return L;
 }
-size_t decode_workspace(const Dims& d) { return decode_layout(d).total; }
+
+// sparse decode: rows_kernel shape (threads per row: enough warps for kRowBatch entries each, up to
+// 1024; CTAs of at least 256 threads when rows are short) and its workspace, in order:
+// acc [B][Hq][kRowSegs][128] fp32, ml [B][Hq][kRowSegs] float2, rowidx [B][Hq][rstride] u32,
+// rlen [B*Hq], arrive [B*Hq], bsum [nb]
+struct SparseLayout {
+    int tpr, rpc, nb, rstride;
+    size_t acc, ml, rowidx, rlen, arrive, bsum, total;
+};
+SparseLayout sparse_layout(const Dims& d) {
+    SparseLayout L;
+    const long rows = (long)d.B * d.Hq;
+    const long need = ((long)d.k_max + kRowBatch - 1) / kRowBatch;   // threads for one pass over a row
+    long tpr = (need + 31) / 32 * 32;
+    if (tpr > 1024) tpr = 1024;
+    L.tpr = (int)tpr;
+    L.rpc = tpr >= 256 ? 1 : (int)(256 / tpr);
+    L.nb = (int)((rows + L.rpc - 1) / L.rpc);
+    L.rstride = (d.k_max + kRowBatch - 1) / kRowBatch * kRowBatch;
+    const size_t slots = (size_t)rows * kRowSegs;
+    L.acc = 0;
+    L.ml = L.acc + align256(slots * kHeadDim * sizeof(float));
+    L.rowidx = L.ml + align256(slots * sizeof(float2));
+    L.rlen = L.rowidx + align256((size_t)rows * L.rstride * sizeof(uint32_t));
+    L.arrive = L.rlen + align256((size_t)rows * sizeof(int));
+    L.bsum = L.arrive + align256((size_t)rows * sizeof(int));
+    L.total = L.bsum + align256((size_t)L.nb * sizeof(int));
+    return L;
+}
+// entries of all rows are counted in int32
+bool sparse_fits(const Dims& d) { return (long)d.B * d.Hq * d.k_max < (1L << 31); }
+size_t decode_workspace(const Dims& d, bool dense) { return dense ? dense_layout(d).total : sparse_layout(d).total; }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -143,12 +173,12 @@ sd_status decode_common(const sd_shape* shape, const void* q, const void* K, con
     if (!aligned(q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(out, 16) || !aligned(workspace, 256) ||
         !aligned(page_table, 4) || !aligned(lens, 4) || (!dense && !aligned(idx, 4)) || !aligned(dev_status, 4))
         return SD_ERR_INVALID_ARG;
-    if (workspace_bytes < decode_workspace(d)) return SD_ERR_WORKSPACE;
+    if (!dense && !sparse_fits(d)) return SD_ERR_UNSUPPORTED;
+    if (workspace_bytes < decode_workspace(d, dense)) return SD_ERR_WORKSPACE;
     DeviceInfo di;
     st = device_info(&di);
     if (st != SD_OK) return st;
-    DecodeArgs a;
-    const DecodeLayout L = decode_layout(d);
+    DecodeArgs a = {};
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     a.q = static_cast<const __nv_bfloat16*>(q);
     a.K = static_cast<const __nv_bfloat16*>(K);
@@ -157,12 +187,6 @@ sd_status decode_common(const sd_shape* shape, const void* q, const void* K, con
     a.lens = lens;
     a.idx = dense ? nullptr : idx;
     a.out = out;
-    a.acc = reinterpret_cast<float*>(ws + L.acc);
-    a.ml = reinterpret_cast<float2*>(ws + L.ml);
-    a.entries = reinterpret_cast<uint2*>(ws + L.entries);
-    a.counts = reinterpret_cast<int*>(ws + L.counts);
-    a.hdr = reinterpret_cast<int*>(ws + L.hdr);
-    a.gtot = a.hdr + 4;
     a.status = dev_status;
     a.B = d.B;
     a.Hq = d.Hq;
@@ -174,19 +198,35 @@ sd_status decode_common(const sd_shape* shape, const void* q, const void* K, con
     a.n_cap = d.n_cap;
     a.nr = d.nr;
     a.nrt = d.nrt;
-    a.jmax = d.jmax;
     int warps = di.sms * di.decode_ctas_per_sm[dense ? 1 : 0][d.G > 8 ? 1 : 0];
     if (warps > kMaxDecodeWarps) warps = kMaxDecodeWarps;
     a.total_warps = warps;   // one warp per CTA
     a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)kHeadDim));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    st = launch_status(launch_prep(a, s));   // zero the row totals the union pass accumulates
-    if (st != SD_OK) return st;
-    st = launch_status(launch_union(a, dense, s));
-    if (st != SD_OK) return st;
-    st = launch_status(launch_decode(a, dense, s));
-    if (st != SD_OK) return st;
-    return launch_status(launch_merge(a, s));
+    if (dense) {
+        const DenseLayout L = dense_layout(d);
+        a.acc = reinterpret_cast<float*>(ws + L.acc);
+        a.ml = reinterpret_cast<float2*>(ws + L.ml);
+        a.counts = reinterpret_cast<int*>(ws + L.counts);
+        a.hdr = reinterpret_cast<int*>(ws + L.hdr);
+        a.gtot = a.hdr + 4;
+        a.jmax = d.jmax;
+        return launch_status(launch_dense(a, s));
+    }
+    const SparseLayout L = sparse_layout(d);
+    a.acc = reinterpret_cast<float*>(ws + L.acc);
+    a.ml = reinterpret_cast<float2*>(ws + L.ml);
+    a.rowidx = reinterpret_cast<uint32_t*>(ws + L.rowidx);
+    a.rlen = reinterpret_cast<int*>(ws + L.rlen);
+    a.arrive = reinterpret_cast<int*>(ws + L.arrive);
+    a.bsum = reinterpret_cast<int*>(ws + L.bsum);
+    a.tpr = L.tpr;
+    a.rpc = L.rpc;
+    a.nb = L.nb;
+    a.rstride = L.rstride;
+    a.jmax = kRowSegs;
+    a.min_epw = (d.k_max + kRowSegs - 2) / (kRowSegs - 1);   // ceil(k_max / (kRowSegs - 1))
+    return launch_status(launch_sparse(a, s));
 }
 
 }  // namespace
@@ -201,7 +241,10 @@ sd_status sd_workspace_size(const sd_shape* shape, int32_t op, size_t* bytes) {
     switch (op) {
         case SD_OP_TOPK: *bytes = topk_workspace(d); return SD_OK;
         case SD_OP_SPARSE:
-        case SD_OP_DENSE: *bytes = decode_workspace(d); return SD_OK;
+            if (!sparse_fits(d)) return SD_ERR_UNSUPPORTED;
+            *bytes = decode_workspace(d, false);
+            return SD_OK;
+        case SD_OP_DENSE: *bytes = decode_workspace(d, true); return SD_OK;
         case SD_OP_QUEST: *bytes = align256((size_t)d.B * d.Hq * d.max_pages * sizeof(float)); return SD_OK;
         default: return SD_ERR_INVALID_ARG;
     }

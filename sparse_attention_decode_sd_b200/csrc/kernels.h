@@ -44,8 +44,10 @@ size_t select_smem(const TopkArgs& a);
 cudaError_t launch_score_pass(const TopkArgs& a, int grid, cudaStream_t stream);
 cudaError_t launch_select(const TopkArgs& a, cudaStream_t stream);
 
-constexpr int kRange = 8192;            // positions per union-building range
+constexpr int kRange = 8192;            // dense decode: positions per counted range
 constexpr int kMaxDecodeWarps = 1280;   // persistent decode warps (one per CTA) at most
+constexpr int kRowSegs = 64;            // sparse decode: segment slots per (b, h) row
+constexpr int kRowBatch = 4;            // sparse decode: consecutive idx entries per rows_kernel thread and pass
 
 struct DecodeArgs {
     const __nv_bfloat16* q;
@@ -55,31 +57,36 @@ struct DecodeArgs {
     const int32_t* lens;
     const int32_t* idx;   // null for dense decode
     float* out;
-    // workspace
-    uint2* entries;       // per range: union rows {cache row index, head mask}, ascending positions
-    int* counts;          // [nrt] union rows per range
-    int* hdr;             // [0] E = all union rows; followed by gtot[B * Hkv], union rows per group
-    int* gtot;            // = hdr + 4 (zeroed together with hdr before the union pass)
+    // workspace, sparse decode
+    uint32_t* rowidx;     // [B*Hq][rstride]: cache row of each idx entry (0xffffffff: none)
+    int* rlen;            // [B*Hq] entries before the first negative one
+    int* arrive;          // [B*Hq] segments of the row finished so far (zeroed by rows_kernel)
+    int* bsum;            // [nb] entries of the rows of each rows_kernel CTA
+    // workspace, dense decode
+    int* counts;          // [nrt] rows per range
+    int* hdr;             // [0] E = all rows; followed by gtot[B * Hkv], rows per group
+    int* gtot;            // = hdr + 4 (zeroed together with hdr before the range pass)
+    // workspace, both
     float2* ml;           // per (b, h, segment) running max (log2 units) and sum
     float* acc;           // per (b, h, segment) un-normalised output [128]
     int32_t* status;
     int B, Hq, Hkv, G, max_pages, num_pages, k_max;
     long n_cap;
-    int nr;               // ranges per (b, kv head) group
-    int nrt;              // B * Hkv * nr
+    int nr;               // dense: ranges per (b, kv head) group
+    int nrt;              // dense: B * Hkv * nr
+    int tpr, rpc, nb;     // sparse: rows_kernel threads per row, rows per CTA, CTAs
+    int rstride;          // sparse: rowidx row stride (k_max rounded up to kRowBatch)
+    int min_epw;          // sparse: entries per warp at least (a row spans <= jmax warps)
     int jmax;             // segment slots per (b, h)
     int total_warps;      // persistent decode warps in the grid
     float scale_log2;     // log2(e) / sqrt(d)
 };
 
 size_t decode_smem();
-size_t union_smem(const DecodeArgs& a);
-// CTAs (one warp each) of the decode kernel variant for (dense, G) that fit on one SM.
+// CTAs (one warp each) of the decode kernel for (dense, G) that fit on one SM.
 cudaError_t decode_occupancy(bool dense, int G, int* ctas_per_sm);
-cudaError_t launch_prep(const DecodeArgs& a, cudaStream_t stream);
-cudaError_t launch_union(const DecodeArgs& a, bool dense, cudaStream_t stream);
-cudaError_t launch_decode(const DecodeArgs& a, bool dense, cudaStream_t stream);
-cudaError_t launch_merge(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_sparse(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_dense(const DecodeArgs& a, cudaStream_t stream);
 
 // Quest page-level indexer.
 constexpr int kQuestMaxPages = 24 * 1024;   // pages per request the page select holds in shared memory

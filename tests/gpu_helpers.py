@@ -36,6 +36,7 @@ class Runner:
         dev = w.q.device
         self.ws_topk = sdb.workspace_for(self.shape, sdb.SD_OP_TOPK, dev)
         self.ws_dec = sdb.workspace_for(self.shape, sdb.SD_OP_SPARSE, dev)
+        self.ws_dense = sdb.workspace_for(self.shape, sdb.SD_OP_DENSE, dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
 
     def topk(self, k=None) -> torch.Tensor:
@@ -54,7 +55,7 @@ class Runner:
     def dense(self) -> torch.Tensor:
         w = self.w
         out = torch.full((w.B, w.Hq, w.d), float("nan"), dtype=torch.float32, device=w.q.device)
-        sdb.sd_dense_decode(self.shape, w.q, w.K, w.V, w.page_table, w.lens, out, self.ws_dec, self.status)
+        sdb.sd_dense_decode(self.shape, w.q, w.K, w.V, w.page_table, w.lens, out, self.ws_dense, self.status)
         return out
 
     def device_status(self) -> int:

@@ -73,11 +73,27 @@ def test_workspace_sizes(lib):
     scores = rows * 8192 * 16 * 4                          # fp32 candidate streams, B*Hq*n_cap
     small = rows * 8192 * 8 + rows * 4 + 3 * 8             # (head, page) records, thresholds, pointers
     assert scores + small <= topk <= scores + small + 4 * 256
+    # sparse decode: 64 segment partials per (b, h) row (fp32 output + max and sum), the cache row of
+    # every idx entry (rows k_max rounded up to 4 entries apart), and per row its length and arrival
+    # counter; then one length sum per CTA of the row pass (1 row per CTA at k_max 2621)
     sparse = sdb.sd_workspace_size(s, sdb.SD_OP_SPARSE)
-    assert sparse == sdb.sd_workspace_size(s, sdb.SD_OP_DENSE)
-    slots = 4 * 64 * (8192 * 16 // 128 + 1)
-    assert sparse >= slots * (128 * 4 + 8)
-    assert sparse % 256 == 0 and topk % 256 == 0
+    need = rows * 64 * (128 * 4 + 8) + rows * 2624 * 4 + rows * 4 * 2 + rows * 4
+    assert need <= sparse <= need + 6 * 256
+    # dense decode: min(N, 1280) + 1 segment partials per (b, h), one row count per 8192 positions of
+    # every (b, KV head) group, and the per-group totals
+    dense = sdb.sd_workspace_size(s, sdb.SD_OP_DENSE)
+    slots = rows * (1280 + 1)
+    need = slots * (128 * 4 + 8) + 4 * 8 * 16 * 4 + (4 + 4 * 8) * 4
+    assert need <= dense <= need + 4 * 256
+    assert sparse % 256 == 0 and dense % 256 == 0 and topk % 256 == 0
+
+
+def test_sparse_workspace_rejects_entry_count_overflow(lib):
+    # B * Hq * k_max entries are counted in int32
+    n = ctypes.c_size_t(0)
+    st = lib.sd_workspace_size(ctypes.byref(_shape(B=64, Hq=128, Hkv=8, k_max=1 << 18, max_pages=1 << 14)),
+                               sdb.SD_OP_SPARSE, ctypes.byref(n))
+    assert st == sdb.SD_ERR_UNSUPPORTED
 
 
 @pytest.mark.parametrize("kw,code", [
