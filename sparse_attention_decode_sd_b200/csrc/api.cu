@@ -199,7 +199,8 @@ sd_status decode_common(const sd_shape* shape, const void* q, const void* K, con
     a.nr = d.nr;
     a.nrt = d.nrt;
     int warps = di.sms * di.decode_ctas_per_sm[dense ? 1 : 0][d.G > 8 ? 1 : 0];
-    if (warps > kMaxDecodeWarps) warps = kMaxDecodeWarps;
+    const int cap = dense ? kMaxDecodeWarps : kMaxSparseWarps;
+    if (warps > cap) warps = cap;
     a.total_warps = warps;   // one warp per CTA
     a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)kHeadDim));
     cudaStream_t s = static_cast<cudaStream_t>(stream);

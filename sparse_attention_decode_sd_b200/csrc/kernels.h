@@ -45,7 +45,8 @@ cudaError_t launch_score_pass(const TopkArgs& a, int grid, cudaStream_t stream);
 cudaError_t launch_select(const TopkArgs& a, cudaStream_t stream);
 
 constexpr int kRange = 8192;            // dense decode: positions per counted range
-constexpr int kMaxDecodeWarps = 1280;   // persistent decode warps (one per CTA) at most
+constexpr int kMaxDecodeWarps = 1280;   // dense decode: persistent warps (one per CTA) at most
+constexpr int kMaxSparseWarps = 4096;   // sparse decode: persistent warps (one per CTA) at most
 constexpr int kRowSegs = 64;            // sparse decode: segment slots per (b, h) row
 constexpr int kRowBatch = 4;            // sparse decode: consecutive idx entries per rows_kernel thread and pass
 
