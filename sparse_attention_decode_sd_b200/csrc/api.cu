@@ -50,8 +50,8 @@ sd_status device_info(DeviceInfo* out) {
 struct Dims {
     int B, Hq, Hkv, G, max_pages, k_max, num_pages;
     long n_cap;   // max_pages * page size
-    int nr;       // dense decode: counted ranges per (b, kv head) group
-    int nrt;      // B * Hkv * nr
+    int nrp;      // dense decode: counted ranges per (b, kv head) group
+    int nrt;      // B * Hkv * nrp
     int jmax;     // dense decode: segment slots per (b, h)
 };
 
@@ -78,7 +78,7 @@ sd_status check_shape(const sd_shape* s, Dims* d) {
     d->k_max = s->k_max;
     d->num_pages = s->num_pages;
     d->n_cap = n_cap;
-    d->nr = (int)nr;
+    d->nrp = (int)nr;
     d->nrt = (int)nrt;
     d->jmax = (int)((n_cap < kMaxDecodeWarps ? n_cap : kMaxDecodeWarps) + 1);
     return SD_OK;
@@ -104,10 +104,9 @@ TopkLayout topk_layout(const Dims& d) {
 }
 size_t topk_workspace(const Dims& d) { return topk_layout(d).total; }
 
-// dense decode workspace, in order: acc [B][Hq][jmax][128] fp32, ml [B][Hq][jmax] float2, counts [nrt],
-// hdr [4] followed by per-group totals [B * Hkv]
+// dense decode workspace, in order: acc [B][Hq][jmax][128] fp32, ml [B][Hq][jmax] float2, counts [nrt]
 struct DenseLayout {
-    size_t acc, ml, counts, hdr, total;
+    size_t acc, ml, counts, total;
 };
 DenseLayout dense_layout(const Dims& d) {
     DenseLayout L;
@@ -115,8 +114,7 @@ DenseLayout dense_layout(const Dims& d) {
     L.acc = 0;
     L.ml = L.acc + align256(slots * kHeadDim * sizeof(float));
     L.counts = L.ml + align256(slots * sizeof(float2));
-    L.hdr = L.counts + align256((size_t)d.nrt * sizeof(int));
-    L.total = L.hdr + align256((4 + (size_t)d.B * d.Hkv) * sizeof(int));
+    L.total = L.counts + align256((size_t)d.nrt * sizeof(int));
     return L;
 }
 
@@ -196,7 +194,7 @@ sd_status decode_common(const sd_shape* shape, const void* q, const void* K, con
     a.num_pages = d.num_pages;
     a.k_max = dense ? 0 : d.k_max;
     a.n_cap = d.n_cap;
-    a.nr = d.nr;
+    a.nrp = d.nrp;
     a.nrt = d.nrt;
     int warps = di.sms * di.decode_ctas_per_sm[dense ? 1 : 0][d.G > 8 ? 1 : 0];
     const int cap = dense ? kMaxDecodeWarps : kMaxSparseWarps;
@@ -209,8 +207,6 @@ sd_status decode_common(const sd_shape* shape, const void* q, const void* K, con
         a.acc = reinterpret_cast<float*>(ws + L.acc);
         a.ml = reinterpret_cast<float2*>(ws + L.ml);
         a.counts = reinterpret_cast<int*>(ws + L.counts);
-        a.hdr = reinterpret_cast<int*>(ws + L.hdr);
-        a.gtot = a.hdr + 4;
         a.jmax = d.jmax;
         return launch_status(launch_dense(a, s));
     }

@@ -44,7 +44,7 @@ size_t select_smem(const TopkArgs& a);
 cudaError_t launch_score_pass(const TopkArgs& a, int grid, cudaStream_t stream);
 cudaError_t launch_select(const TopkArgs& a, cudaStream_t stream);
 
-constexpr int kRange = 8192;            // dense decode: positions per counted range
+constexpr int kRange = 16384;           // dense decode: positions per counted range
 constexpr int kMaxDecodeWarps = 1280;   // dense decode: persistent warps (one per CTA) at most
 constexpr int kMaxSparseWarps = 4096;   // sparse decode: persistent warps (one per CTA) at most
 constexpr int kRowSegs = 64;            // sparse decode: segment slots per (b, h) row
@@ -65,16 +65,14 @@ struct DecodeArgs {
     int* bsum;            // [nb] entries of the rows of each rows_kernel CTA
     // workspace, dense decode
     int* counts;          // [nrt] rows per range
-    int* hdr;             // [0] E = all rows; followed by gtot[B * Hkv], rows per group
-    int* gtot;            // = hdr + 4 (zeroed together with hdr before the range pass)
     // workspace, both
     float2* ml;           // per (b, h, segment) running max (log2 units) and sum
     float* acc;           // per (b, h, segment) un-normalised output [128]
     int32_t* status;
     int B, Hq, Hkv, G, max_pages, num_pages, k_max;
     long n_cap;
-    int nr;               // dense: ranges per (b, kv head) group
-    int nrt;              // dense: B * Hkv * nr
+    int nrp;              // dense: ranges per (b, kv head) group
+    int nrt;              // dense: B * Hkv * nrp
     int tpr, rpc, nb;     // sparse: rows_kernel threads per row, rows per CTA, CTAs
     int rstride;          // sparse: rowidx row stride (k_max rounded up to kRowBatch)
     int min_epw;          // sparse: entries per warp at least (a row spans <= jmax warps)

@@ -25,10 +25,11 @@
 //                         warp stores its (max, sum, output) partial and the last of the row's warps to
 //                         arrive (a counter per row) merges the partials by log-sum-exp.
 //
-// Dense decode (the comparator), four kernels: prep_kernel zeroes the row totals; ranges_kernel counts
-// the positions of each 8192-position range of every (request, KV head) group; dense_decode_kernel
-// walks all rows of every group with the same tile pipeline, one 16-row tile serving all G heads of
-// the group (S = K_tile . Q^T with the G heads as columns); merge_kernel combines the segment partials.
+// Dense decode (the comparator), three kernels: ranges_kernel counts the positions of each
+// kRange-position range of every (request, KV head) group; dense_decode_kernel walks all rows of every
+// group with the same tile pipeline, one 16-row tile serving all G heads of the group (S = K_tile . Q^T
+// with the G heads as columns), its first range found from the counts; merge_kernel (four warps per
+// (b, h)) combines the segment partials.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -39,7 +40,6 @@ constexpr int kTileRows = 16;
 constexpr int kRowPitch = kRowBytes + 16;   // padded shared-memory row: ldmatrix phases hit 8 distinct bank groups
 constexpr int kTileBytes = kTileRows * kRowPitch;
 constexpr int kFlagFirst = 1, kFlagLast = 2, kFlagEnd = 4;
-constexpr int kRangeThreads = 256;
 constexpr uint32_t kNoRow = 0xffffffffu;    // rowidx entry of a position that maps to no cache row
 constexpr int kPrologue = 8;                // length sums per lane loaded together by a decode warp
 
@@ -573,25 +573,18 @@ __global__ void __launch_bounds__(32) sparse_decode_kernel(DecodeArgs a) {
 // ---------------------------------------------------------------------------------------------
 // dense decode: ranges_kernel, dense_decode_kernel, merge_kernel
 // ---------------------------------------------------------------------------------------------
-// One CTA per 8192-position range of each group: the range's row count, added to the group and
-// global totals (zeroed by prep_kernel).
-__global__ void __launch_bounds__(kRangeThreads) ranges_kernel(DecodeArgs a) {
+// Dense decode: the row count of each range (every position below N_b is a row).
+__global__ void __launch_bounds__(256) ranges_kernel(DecodeArgs a) {
     pdl_enter();
-    if (threadIdx.x != 0) return;
-    const int ri = blockIdx.x;
-    const int grp = ri / a.nr, r = ri - grp * a.nr;
-    const int b = grp / a.Hkv;
-    const int n = checked_len(a.lens, b, a.n_cap, a.status);
-    const int lo = r * kRange, hi = min(lo + kRange, n);
-    const int cnt = lo < hi ? hi - lo : 0;
-    a.counts[ri] = cnt;
-    if (cnt > 0) {
-        atomicAdd(&a.gtot[grp], cnt);
-        atomicAdd(&a.hdr[0], cnt);
-    }
+    const int ri = blockIdx.x * blockDim.x + threadIdx.x;
+    if (ri >= a.nrt) return;
+    const int grp = ri / a.nrp, rloc = ri - grp * a.nrp;
+    const int n = checked_len(a.lens, grp / a.Hkv, a.n_cap, a.status);
+    const int lo = rloc * kRange;
+    a.counts[ri] = lo < n ? min(kRange, n - lo) : 0;
 }
 
-// The warp's walk over the rows of the groups (all fields warp-uniform).
+// The warp's walk over its rows (all fields warp-uniform).
 struct GroupWalker {
     int e, e_end;     // next global row and the end of this warp's share
     int ri, off;      // range holding row e, and e's offset in it
@@ -599,8 +592,19 @@ struct GroupWalker {
     int grp;          // group (b * Hkv + kvh) of the current segment
     int seg_j;        // segment slot of the current segment
     bool seg_new;     // the next tile opens a segment
-    int epw;
+    int epw;          // rows per warp
 };
+
+// The next non-empty range after ri (one exists while rows remain; at the last range *cnt = 0).
+__device__ __forceinline__ int next_range(const DecodeArgs& a, int ri, int* cnt) {
+    int c = 0;
+    while (ri + 1 < a.nrt) {
+        c = __ldg(a.counts + (++ri));
+        if (c != 0) break;
+    }
+    *cnt = c;
+    return ri;
+}
 
 __device__ __forceinline__ TileDesc prefetch_group_tile(const DecodeArgs& a, GroupWalker& w) {
     const int lane = threadIdx.x & 31;
@@ -619,26 +623,29 @@ __device__ __forceinline__ TileDesc prefetch_group_tile(const DecodeArgs& a, Gro
     int filled = 0;
     while (filled < kTileRows && w.e < w.e_end) {
         if (w.off == w.cnt) {   // next non-empty range; stop at a group boundary
-            int ri = w.ri + 1;
-            int c = __ldg(a.counts + ri);
-            while (c == 0) c = __ldg(a.counts + (++ri));
-            if (ri / a.nr != grp) break;
+            int c;
+            const int ri = next_range(a, w.ri, &c);
+            if (ri / a.nrp != grp) break;
             w.ri = ri;
             w.off = 0;
             w.cnt = c;
         }
         const int take = min(min(kTileRows - filled, w.cnt - w.off), w.e_end - w.e);
+        if (take <= 0) {   // not reached (counts are consistent); ends the walk
+            w.e = w.e_end;
+            break;
+        }
         if (lane >= filled && lane < filled + take) {
-            const int p = (w.ri - grp * a.nr) * kRange + w.off + lane - filled;
-            int page = __ldg(a.page_table + (long)b * a.max_pages + p / kPageSize);
-            uint32_t m = full_mask;
+            const int off = w.off + lane - filled;
+            const int p = (w.ri - grp * a.nrp) * kRange + off;
+            const int page = __ldg(a.page_table + (long)b * a.max_pages + p / kPageSize);
             if (page < 0 || page >= a.num_pages) {
                 report(a.status, SD_ERR_INDEX_OOB);
-                page = 0;
-                m = 0;
+                d.row_idx = kNoRow;
+            } else {
+                d.row_idx = ((uint32_t)page * kPageSize + (uint32_t)(p & (kPageSize - 1))) * (uint32_t)a.Hkv + kvh;
             }
-            d.row_idx = ((uint32_t)page * kPageSize + (uint32_t)(p & (kPageSize - 1))) * (uint32_t)a.Hkv + kvh;
-            d.mask = m;
+            d.mask = full_mask;
         }
         filled += take;
         w.off += take;
@@ -648,15 +655,14 @@ __device__ __forceinline__ TileDesc prefetch_group_tile(const DecodeArgs& a, Gro
     // does the segment end here?
     bool last = w.e >= w.e_end;
     if (!last && w.off == w.cnt) {
-        int ri = w.ri + 1;
-        int c = __ldg(a.counts + ri);
-        while (c == 0) c = __ldg(a.counts + (++ri));
-        if (ri / a.nr != grp) {
+        int c;
+        const int ri = next_range(a, w.ri, &c);
+        if (ri / a.nrp != grp) {
             last = true;
             w.ri = ri;   // the next segment starts in range ri
             w.off = 0;
             w.cnt = c;
-            w.grp = ri / a.nr;
+            w.grp = ri / a.nrp;
             w.seg_j = (int)(blockIdx.x - w.e / w.epw);   // w.e is the first row of the new group
             w.seg_new = true;
         }
@@ -708,6 +714,23 @@ __device__ __forceinline__ void flush_group(const DecodeArgs& a, int b, int kvh,
     }
 }
 
+// Sum of the range counts [lo, hi), kPrologue loads per lane in flight (warp-uniform result).
+__device__ __forceinline__ int sum_counts(const DecodeArgs& a, int lo, int hi) {
+    const int lane = threadIdx.x & 31;
+    int s = 0;
+    for (int base = lo; base < hi; base += 32 * kPrologue) {
+        int v[kPrologue];
+#pragma unroll
+        for (int i = 0; i < kPrologue; ++i) {
+            const int k = base + 32 * i + lane;
+            v[i] = k < hi ? __ldg(a.counts + k) : 0;
+        }
+#pragma unroll
+        for (int i = 0; i < kPrologue; ++i) s += v[i];
+    }
+    return __reduce_add_sync(0xffffffffu, s);
+}
+
 template <int NT>
 __global__ void __launch_bounds__(32) dense_decode_kernel(DecodeArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
@@ -715,46 +738,44 @@ __global__ void __launch_bounds__(32) dense_decode_kernel(DecodeArgs a) {
     pdl_enter();
 
     const int lane = threadIdx.x & 31;
-    const int E = a.hdr[0];
+    const int E = sum_counts(a, 0, a.nrt);
     if (E == 0) return;
     GroupWalker w;
     w.epw = max(1, (int)(((long)E + a.total_warps - 1) / a.total_warps));
-    w.e = (int)blockIdx.x * w.epw;
-    if (w.e >= E) return;
-    w.e_end = min(E, w.e + w.epw);
-    // the group holding row w.e (prefix over the per-group totals), then its range
-    int e0grp = 0;
-    w.grp = -1;
+    const long e0 = (long)blockIdx.x * w.epw;
+    if (e0 >= E) return;
+    w.e = (int)e0;
+    w.e_end = (int)min((long)E, e0 + w.epw);
+    // the range holding row w.e (prefix over the counts, kPrologue loads per lane in flight)
+    int ri = -1, ri0 = 0;
     {
-        const int ngroups = a.B * a.Hkv;
         int acc = 0;
-        for (int base = 0; base < ngroups && w.grp < 0; base += 32) {
-            const int v = (base + lane < ngroups) ? __ldg(a.gtot + base + lane) : 0;
-            const int incl = warp_inclusive_scan(v);
-            const int tot = __shfl_sync(0xffffffffu, incl, 31);
-            if (w.e < acc + tot) {
-                const int l = __ffs(__ballot_sync(0xffffffffu, acc + incl > w.e)) - 1;
-                w.grp = base + l;
-                e0grp = acc + __shfl_sync(0xffffffffu, incl - v, l);
+        for (int base = 0; base < a.nrt && ri < 0; base += 32 * kPrologue) {
+            int v[kPrologue];
+#pragma unroll
+            for (int i = 0; i < kPrologue; ++i) {
+                const int k = base + 32 * i + lane;
+                v[i] = k < a.nrt ? __ldg(a.counts + k) : 0;
             }
-            acc += tot;
-        }
-        const int off_g = w.e - e0grp;
-        int acc2 = 0;
-        w.ri = -1;
-        for (int base = 0; base < a.nr && w.ri < 0; base += 32) {
-            const int v = (base + lane < a.nr) ? __ldg(a.counts + w.grp * a.nr + base + lane) : 0;
-            const int incl = warp_inclusive_scan(v);
-            const int tot = __shfl_sync(0xffffffffu, incl, 31);
-            if (off_g < acc2 + tot) {
-                const int l = __ffs(__ballot_sync(0xffffffffu, acc2 + incl > off_g)) - 1;
-                w.ri = w.grp * a.nr + base + l;
-                w.off = off_g - (acc2 + __shfl_sync(0xffffffffu, incl - v, l));
+#pragma unroll
+            for (int i = 0; i < kPrologue; ++i) {
+                const int incl = warp_inclusive_scan(v[i]);
+                const uint32_t hit = __ballot_sync(0xffffffffu, acc + incl > w.e);
+                if (ri < 0 && hit != 0u) {
+                    const int l = __ffs(hit) - 1;
+                    ri = base + 32 * i + l;
+                    ri0 = acc + __shfl_sync(0xffffffffu, incl - v[i], l);
+                }
+                acc += __shfl_sync(0xffffffffu, incl, 31);
             }
-            acc2 += tot;
         }
     }
-    w.cnt = __ldg(a.counts + w.ri);
+    if (ri < 0) return;   // not reached: w.e < E
+    w.ri = ri;
+    w.off = w.e - ri0;
+    w.cnt = __ldg(a.counts + ri);
+    w.grp = ri / a.nrp;
+    const int e0grp = ri0 - sum_counts(a, w.grp * a.nrp, ri);   // first row of the group
     w.seg_j = (int)(blockIdx.x - e0grp / w.epw);
     w.seg_new = true;
 
@@ -768,6 +789,7 @@ __global__ void __launch_bounds__(32) dense_decode_kernel(DecodeArgs a) {
     }
     for (int t = 0;; ++t) {
         const int stage = t % kStages;
+        // the stage of tile t-1 is free: issue tile t+kStages-1 before waiting for tile t
         issue_tile(a, ws, (t + kStages - 1) % kStages, next);
         next = prefetch_group_tile(a, w);
         cp_async_wait<kStages - 1>();
@@ -787,73 +809,103 @@ __global__ void __launch_bounds__(32) dense_decode_kernel(DecodeArgs a) {
     cp_async_wait<0>();
 }
 
-// One CTA per (b, h), one thread per output dimension: log-sum-exp merge of the segment partials of
-// its group, 32 segments at a time (all loads of a chunk are in flight together).
-__global__ void __launch_bounds__(kHeadDim) merge_kernel(DecodeArgs a) {
-    __shared__ float s_m[32];   // per-segment weights of the current chunk
-    __shared__ float s_l[32];
-    __shared__ float s_scale[1];
+// ---------------------------------------------------------------------------------------------
+// dense decode: merge_kernel
+// ---------------------------------------------------------------------------------------------
+constexpr int kMergeWarps = 4;
+constexpr int kMergeLoads = 16;   // partials per lane whose loads are in flight together
+
+// One CTA of kMergeWarps warps per (b, h): log-sum-exp merge of the partials of the segments of its
+// group.  Every thread takes segments t, t + 128, ... for the maxima and weights; warp w then sums the
+// outputs of segments w, w + kMergeWarps, ... (lane l owns dimensions 4l .. 4l+3), and the warps' sums
+// are added in shared memory.
+__global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(DecodeArgs a) {
+    __shared__ float s_red[kMergeWarps];
+    __shared__ float4 s_o[kMergeWarps][32];
     pdl_enter();
-    const int d = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const long bh = blockIdx.x;
-    const int b = (int)(bh / a.Hq), h = (int)(bh % a.Hq), kvh = h / a.G;
-    __shared__ int s_e0;
-    const int grp = b * a.Hkv + kvh;
-    if (d < 32) {   // first row of the group: prefix over the per-group totals
-        int acc = 0;
-        for (int base = 0; base < grp; base += 32) {
-            int v = (base + d < grp) ? a.gtot[base + d] : 0;
+    const int b = (int)(bh / a.Hq), h = (int)(bh % a.Hq);
+    const int grp = b * a.Hkv + h / a.G;
+    // all rows, the rows of the groups before this one and this group's rows, in one pass over the counts
+    int E = 0, e0 = 0, eg = 0;
+    {
+        const int g0 = grp * a.nrp, g1 = g0 + a.nrp;
+        for (int base = 0; base < a.nrt; base += 32 * kPrologue) {
+            int v[kPrologue];
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-            acc += v;
+            for (int i = 0; i < kPrologue; ++i) {
+                const int k = base + 32 * i + lane;
+                v[i] = k < a.nrt ? __ldg(a.counts + k) : 0;
+            }
+#pragma unroll
+            for (int i = 0; i < kPrologue; ++i) {
+                const int k = base + 32 * i + lane;
+                E += v[i];
+                e0 += k < g0 ? v[i] : 0;
+                eg += (k >= g0 && k < g1) ? v[i] : 0;
+            }
         }
-        if (d == 0) s_e0 = acc;
+        E = __reduce_add_sync(0xffffffffu, E);
+        e0 = __reduce_add_sync(0xffffffffu, e0);
+        eg = __reduce_add_sync(0xffffffffu, eg);
     }
-    __syncthreads();
-    const int E = a.hdr[0];
+    const int e1 = e0 + eg;
     const int epw = max(1, (int)(((long)E + a.total_warps - 1) / a.total_warps));
-    const int e0 = s_e0, e1 = e0 + a.gtot[grp];
     const int nseg = (e1 > e0) ? ((e1 - 1) / epw - e0 / epw + 1) : 0;
     const float2* ml = a.ml + bh * a.jmax;
-    const float* accp = a.acc + bh * a.jmax * kHeadDim + d;
-    float M = -INFINITY, L = 0.f, o = 0.f;
-    for (int j0 = 0; j0 < nseg; j0 += 32) {
-        const int cnt = min(32, nseg - j0);
-        float x[32];
+    // M = max over the segments' maxima
+    float mx = -INFINITY;
+    for (int j = tid; j < nseg; j += blockDim.x) mx = fmaxf(mx, ml[j].x);
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) x[jj] = (jj < cnt) ? accp[(long)(j0 + jj) * kHeadDim] : 0.f;
-        if (d < 32) {   // warp 0: the chunk's max, then one weight per segment
-            const float2 v = (d < cnt) ? ml[j0 + d] : make_float2(-INFINITY, 0.f);
-            float cm = v.x;
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (lane == 0) s_red[warp] = mx;
+    __syncthreads();
+    float M = s_red[0];
 #pragma unroll
-            for (int o2 = 16; o2 > 0; o2 >>= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, o2));
-            const float nm = fmaxf(M, cm);
-            s_m[d] = (v.x == -INFINITY) ? 0.f : exp2f(v.x - nm);   // weight of segment j0 + d
-            s_l[d] = v.y;
-            if (d == 0) s_scale[0] = nm;
+    for (int w = 1; w < kMergeWarps; ++w) M = fmaxf(M, s_red[w]);
+    __syncthreads();
+    // warp `warp` sums segments warp, warp + kMergeWarps, ...
+    float L = 0.f;
+    float4 o4 = make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4* src = reinterpret_cast<const float4*>(a.acc + bh * a.jmax * kHeadDim) + lane;
+    for (int j0 = warp; j0 < nseg; j0 += kMergeWarps * kMergeLoads) {
+        float4 x[kMergeLoads];
+        float2 v[kMergeLoads];
+#pragma unroll
+        for (int i = 0; i < kMergeLoads; ++i) {   // unconditional (clamped) loads, all in flight together
+            const int j = min(j0 + i * kMergeWarps, nseg - 1);
+            x[i] = __ldg(src + (long)j * (kHeadDim / 4));
+            v[i] = __ldg(ml + j);
         }
-        __syncthreads();
-        const float nm = s_scale[0];
-        if (nm != -INFINITY) {
-            const float sc = (M == -INFINITY) ? 0.f : exp2f(M - nm);
-            o *= sc;
-            L *= sc;
 #pragma unroll
-            for (int jj = 0; jj < 32; ++jj) {
-                o += s_m[jj] * x[jj];
-                L += s_m[jj] * s_l[jj];
-            }
-            M = nm;
+        for (int i = 0; i < kMergeLoads; ++i) {
+            const bool live = j0 + i * kMergeWarps < nseg;
+            const float wj = (!live || v[i].x == -INFINITY) ? 0.f : exp2f(v[i].x - M);
+            L += wj * v[i].y;
+            o4.x += wj * x[i].x;
+            o4.y += wj * x[i].y;
+            o4.z += wj * x[i].z;
+            o4.w += wj * x[i].w;
         }
-        __syncthreads();
     }
-    a.out[bh * kHeadDim + d] = L > 0.f ? o / L : 0.f;
-}
-
-// Zeroes the per-group and global row totals that ranges_kernel accumulates.
-__global__ void __launch_bounds__(256) prep_kernel(DecodeArgs a) {
-    pdl_enter();
-    for (int i = threadIdx.x; i < 4 + a.B * a.Hkv; i += blockDim.x) a.hdr[i] = 0;
+    s_o[warp][lane] = o4;
+    if (lane == 0) s_red[warp] = L;
+    __syncthreads();
+    if (warp == 0) {
+        float Lt = 0.f;
+        float4 ot = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int w = 0; w < kMergeWarps; ++w) {
+            Lt += s_red[w];
+            ot.x += s_o[w][lane].x;
+            ot.y += s_o[w][lane].y;
+            ot.z += s_o[w][lane].z;
+            ot.w += s_o[w][lane].w;
+        }
+        const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
+        reinterpret_cast<float4*>(a.out + bh * kHeadDim)[lane] = make_float4(ot.x * inv, ot.y * inv, ot.z * inv, ot.w * inv);
+    }
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -880,15 +932,13 @@ cudaError_t launch_sparse(const DecodeArgs& a, cudaStream_t stream) {
 }
 
 cudaError_t launch_dense(const DecodeArgs& a, cudaStream_t stream) {
-    cudaError_t e = launch_pdl(prep_kernel, dim3(1), dim3(256), 0, stream, a);
-    if (e != cudaSuccess) return e;
-    e = launch_pdl(ranges_kernel, dim3(a.nrt), dim3(kRangeThreads), 0, stream, a);
+    cudaError_t e = launch_pdl(ranges_kernel, dim3((unsigned)((a.nrt + 255) / 256)), dim3(256), 0, stream, a);
     if (e != cudaSuccess) return e;
     const dim3 grid(a.total_warps), block(32);
     e = a.G <= 8 ? launch_pdl(dense_decode_kernel<1>, grid, block, decode_smem(), stream, a)
                  : launch_pdl(dense_decode_kernel<2>, grid, block, decode_smem(), stream, a);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(merge_kernel, dim3((unsigned)((long)a.B * a.Hq)), dim3(kHeadDim), 0, stream, a);
+    e = launch_pdl(merge_kernel, dim3((unsigned)((long)a.B * a.Hq)), dim3(kMergeWarps * 32), 0, stream, a);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 

@@ -79,12 +79,12 @@ def test_workspace_sizes(lib):
     sparse = sdb.sd_workspace_size(s, sdb.SD_OP_SPARSE)
     need = rows * 64 * (128 * 4 + 8) + rows * 2624 * 4 + rows * 4 * 2 + rows * 4
     assert need <= sparse <= need + 6 * 256
-    # dense decode: min(N, 1280) + 1 segment partials per (b, h), one row count per 8192 positions of
-    # every (b, KV head) group, and the per-group totals
+    # dense decode: min(N, 1280) + 1 segment partials per (b, h) and one row count per 16384 positions
+    # of every (b, KV head) group
     dense = sdb.sd_workspace_size(s, sdb.SD_OP_DENSE)
     slots = rows * (1280 + 1)
-    need = slots * (128 * 4 + 8) + 4 * 8 * 16 * 4 + (4 + 4 * 8) * 4
-    assert need <= dense <= need + 4 * 256
+    need = slots * (128 * 4 + 8) + 4 * 8 * 8 * 4
+    assert need <= dense <= need + 3 * 256
     assert sparse % 256 == 0 and dense % 256 == 0 and topk % 256 == 0
 
 
