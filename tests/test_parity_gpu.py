@@ -44,6 +44,7 @@ SMALL = [
     (4, 8, 2, [0, 15, 16, 17], [3, 20, 1, 5], "shuffled"),  # empty context, k > N, N < 16
     (1, 8, 1, [20000], [1], "shuffled"),                    # k = 1
     (1, 8, 2, [9000], [9000 // 3], "shuffled"),             # dense-ish selection (k = N/3)
+    (1, 256, 16, [700], [30], "shuffled"),                  # the most heads supported: Hkv = 16, G = 16
 ]
 
 
