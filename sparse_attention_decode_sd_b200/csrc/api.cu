@@ -66,7 +66,8 @@ sd_status check_shape(const sd_shape* s, Dims* d) {
     if (G > kMaxGroup || s->num_kv_heads > 16 || s->batch > kMaxBatch) return SD_ERR_UNSUPPORTED;
     const long n_cap = (long)s->max_pages_per_req * kPageSize;
     if (n_cap > (1L << 30)) return SD_ERR_UNSUPPORTED;
-    if ((long)s->num_pages * kPageSize * s->num_kv_heads >= (1L << 32)) return SD_ERR_UNSUPPORTED;   // row index is 32-bit
+    // cache rows are indexed in 32 bits, and as signed TMA coordinates by the sparse decode
+    if ((long)s->num_pages * kPageSize * s->num_kv_heads >= (1L << 31)) return SD_ERR_UNSUPPORTED;
     const long nr = (n_cap + kRange - 1) / kRange;
     const long nrt = (long)s->batch * s->num_kv_heads * nr;
     if (nrt * kRange >= (1L << 31)) return SD_ERR_UNSUPPORTED;   // rows are counted in int32
@@ -120,11 +121,10 @@ DenseLayout dense_layout(const Dims& d) {
 
 // sparse decode: rows_kernel shape (threads per row: enough warps for kRowBatch entries each, up to
 // 1024; CTAs of at least 256 threads when rows are short) and its workspace, in order:
-// acc [B][Hq][kRowSegs][128] fp32, ml [B][Hq][kRowSegs] float2, rowidx [B][Hq][rstride] u32,
-// rlen [B*Hq], arrive [B*Hq], bsum [nb]
+// acc [B][Hq][kRowSegs][128] fp32, ml [B][Hq][kRowSegs] float2, rlen [B*Hq], arrive [B*Hq], bsum [nb]
 struct SparseLayout {
-    int tpr, rpc, nb, rstride;
-    size_t acc, ml, rowidx, rlen, arrive, bsum, total;
+    int tpr, rpc, nb;
+    size_t acc, ml, rlen, arrive, bsum, total;
 };
 SparseLayout sparse_layout(const Dims& d) {
     SparseLayout L;
@@ -135,12 +135,10 @@ SparseLayout sparse_layout(const Dims& d) {
     L.tpr = (int)tpr;
     L.rpc = tpr >= 256 ? 1 : (int)(256 / tpr);
     L.nb = (int)((rows + L.rpc - 1) / L.rpc);
-    L.rstride = (d.k_max + kRowBatch - 1) / kRowBatch * kRowBatch;
     const size_t slots = (size_t)rows * kRowSegs;
     L.acc = 0;
     L.ml = L.acc + align256(slots * kHeadDim * sizeof(float));
-    L.rowidx = L.ml + align256(slots * sizeof(float2));
-    L.rlen = L.rowidx + align256((size_t)rows * L.rstride * sizeof(uint32_t));
+    L.rlen = L.ml + align256(slots * sizeof(float2));
     L.arrive = L.rlen + align256((size_t)rows * sizeof(int));
     L.bsum = L.arrive + align256((size_t)rows * sizeof(int));
     L.total = L.bsum + align256((size_t)L.nb * sizeof(int));
@@ -213,14 +211,12 @@ sd_status decode_common(const sd_shape* shape, const void* q, const void* K, con
     const SparseLayout L = sparse_layout(d);
     a.acc = reinterpret_cast<float*>(ws + L.acc);
     a.ml = reinterpret_cast<float2*>(ws + L.ml);
-    a.rowidx = reinterpret_cast<uint32_t*>(ws + L.rowidx);
     a.rlen = reinterpret_cast<int*>(ws + L.rlen);
     a.arrive = reinterpret_cast<int*>(ws + L.arrive);
     a.bsum = reinterpret_cast<int*>(ws + L.bsum);
     a.tpr = L.tpr;
     a.rpc = L.rpc;
     a.nb = L.nb;
-    a.rstride = L.rstride;
     a.jmax = kRowSegs;
     a.min_epw = (d.k_max + kRowSegs - 2) / (kRowSegs - 1);   // ceil(k_max / (kRowSegs - 1))
     return launch_status(launch_sparse(a, s));

@@ -59,7 +59,6 @@ struct DecodeArgs {
     const int32_t* idx;   // null for dense decode
     float* out;
     // workspace, sparse decode
-    uint32_t* rowidx;     // [B*Hq][rstride]: cache row of each idx entry (0xffffffff: none)
     int* rlen;            // [B*Hq] entries before the first negative one
     int* arrive;          // [B*Hq] segments of the row finished so far (zeroed by rows_kernel)
     int* bsum;            // [nb] entries of the rows of each rows_kernel CTA
@@ -74,7 +73,6 @@ struct DecodeArgs {
     int nrp;              // dense: ranges per (b, kv head) group
     int nrt;              // dense: B * Hkv * nrp
     int tpr, rpc, nb;     // sparse: rows_kernel threads per row, rows per CTA, CTAs
-    int rstride;          // sparse: rowidx row stride (k_max rounded up to kRowBatch)
     int min_epw;          // sparse: entries per warp at least (a row spans <= jmax warps)
     int jmax;             // segment slots per (b, h)
     int total_warps;      // persistent decode warps in the grid
@@ -82,6 +80,7 @@ struct DecodeArgs {
 };
 
 size_t decode_smem();
+size_t sparse_decode_smem();
 // CTAs (one warp each) of the decode kernel for (dense, G) that fit on one SM.
 cudaError_t decode_occupancy(bool dense, int G, int* ctas_per_sm);
 cudaError_t launch_sparse(const DecodeArgs& a, cudaStream_t stream);

@@ -6,41 +6,50 @@
 // Sparse decode, two kernels per call:
 //   rows_kernel           one group of threads per (request, query head) row of idx: checks the row
 //                         (ascending positions below N_b, then negative padding only), finds its length
-//                         (the index of the first negative entry), maps every position to its cache row
-//                         through the page table, zeroes the output of empty rows and the row's arrival
-//                         counter, and writes per-CTA length sums.
-//   sparse_decode_kernel  one warp per CTA, a persistent grid of one wave.  The selected entries of all
-//                         rows, in (request, head, position) order, are cut evenly across the warps; a
-//                         warp finds its first row from the length sums and streams its entries in
-//                         tiles of 16 rows: 16-byte cp.async gathers of the 256-byte K and V rows into
-//                         272-byte padded shared-memory rows, three tiles in flight.  The heads of a GQA
-//                         group are consecutive rows, so their warps run side by side and a row several
-//                         of them selected is mostly served from L2 after its first read.  On the tensor
-//                         cores (mma.sync m16n8k16, bf16 in, fp32 accumulate), with q in column 0 of the
-//                         B operand:
-//                             S   = K_tile (16 rows x 128) . q                  8 MMAs
-//                             o  += V_tile^T (128 x 16 rows) . p                16 MMAs (p as bf16 hi + lo)
-//                         and an fp32 online softmax in between.  A warp's part of one row is a
-//                         "segment": a row held by one warp is written out directly; otherwise each
-//                         warp stores its (max, sum, output) partial and the last of the row's warps to
-//                         arrive (a counter per row) merges the partials by log-sum-exp.
+//                         (the index of the first negative entry), zeroes the output of empty rows and
+//                         the row's arrival counter, and writes per-CTA length sums.
+//   sparse_decode_kernel  one warp per CTA, a persistent grid of one wave (12 warps per SM).  The
+//                         selected entries of all rows, in (request, head, position) order, are cut
+//                         evenly across the warps; a warp finds its first row from the length sums and
+//                         streams its entries in tiles of 16 rows.  Per tile, in a software pipeline
+//                         that waits for no load but the gather itself: the positions are loaded four
+//                         tiles ahead, mapped through the page table two tiles ahead, and the 256-byte
+//                         K and V rows gathered one tile ahead by TMA four-row gathers (tile::gather4,
+//                         64-dim halves with the 128-byte swizzle) into a two-stage shared-memory ring.
+//                         The heads of a GQA group are consecutive rows, so their warps run side by side
+//                         and a row several of them selected is mostly served from L2 after its first
+//                         read.  On the tensor cores (mma.sync m16n8k16, bf16 in, fp32 accumulate):
+//                             S   = K_tile (16 rows x 128) . q              8 MMAs (q: column 0 of B)
+//                             o  += V_tile^T (128 x 16 rows) . [p_hi, p_lo] 8 MMAs (columns 0 and 1 of B)
+//                         with an fp32 online softmax in between; the weights p enter as a bf16 high
+//                         part and a bf16 residual, and the head's output is the sum of the two
+//                         accumulator columns.  A warp's part of one row is a "segment": a row held by
+//                         one warp is written out directly; otherwise each warp stores its (max, sum,
+//                         output) partial and the last of the row's warps to arrive (a counter per
+//                         row) merges the partials by log-sum-exp.
 //
 // Dense decode (the comparator), three kernels: ranges_kernel counts the positions of each
 // kRange-position range of every (request, KV head) group; dense_decode_kernel walks all rows of every
 // group with the same tile pipeline, one 16-row tile serving all G heads of the group (S = K_tile . Q^T
 // with the G heads as columns), its first range found from the counts; merge_kernel (four warps per
 // (b, h)) combines the segment partials.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.h"
 
 namespace sd {
 
-constexpr int kStages = 3;                  // tiles in flight per decode warp
+constexpr int kStages = 3;                  // tiles in flight per dense decode warp
+constexpr int kSparseStages = 2;            // tiles in flight per sparse decode warp
 constexpr int kTileRows = 16;
 constexpr int kRowPitch = kRowBytes + 16;   // padded shared-memory row: ldmatrix phases hit 8 distinct bank groups
 constexpr int kTileBytes = kTileRows * kRowPitch;
 constexpr int kFlagFirst = 1, kFlagLast = 2, kFlagEnd = 4;
-constexpr uint32_t kNoRow = 0xffffffffu;    // rowidx entry of a position that maps to no cache row
+constexpr uint32_t kNoRow = 0xffffffffu;    // cache row of a position that maps to none (dense decode)
 constexpr int kPrologue = 8;                // length sums per lane loaded together by a decode warp
 
 // ---------------------------------------------------------------------------------------------
@@ -252,7 +261,10 @@ __device__ __forceinline__ int warp_inclusive_scan(int v) {
 // One group of a.tpr threads (whole warps) per row, a.rpc rows per CTA.  Each thread takes kRowBatch
 // consecutive entries per pass (the whole row in one pass when k_max <= kRowBatch * tpr), so
 // consecutive lanes hold consecutive runs and an entry's predecessor is in the same thread or the
-// lane before.  rowidx rows are a.rstride (a multiple of kRowBatch) entries apart.
+// lane before.  Checks the row (ascending positions below N_b, then negative padding only), finds
+// its length (the index of the first negative entry), zeroes the output of empty rows and the
+// row's arrival counter, and writes per-CTA length sums.  Positions are mapped to cache rows by the
+// decode kernel itself, as it streams.
 __global__ void __launch_bounds__(1024, 2) rows_kernel(DecodeArgs a) {
     __shared__ int s_neg[32];   // per warp: first negative entry it saw
     __shared__ int s_len[32];   // per row of this CTA
@@ -265,11 +277,9 @@ __global__ void __launch_bounds__(1024, 2) rows_kernel(DecodeArgs a) {
     const int k_max = a.k_max;
     int first_neg = k_max;
     if (r < R) {   // uniform over the row's warps
-        const int b = r / a.Hq, kvh = (r - b * a.Hq) / a.G;
+        const int b = r / a.Hq;
         const int n = checked_len(a.lens, b, a.n_cap, a.status);
         const int32_t* row = a.idx + (long)r * k_max;
-        uint32_t* dst = a.rowidx + (long)r * a.rstride;
-        const int32_t* ptrow = a.page_table + (long)b * a.max_pages;
         for (int base = 0; base < k_max; base += tpr * kRowBatch) {   // uniform over the row's threads
             const int j0 = base + t * kRowBatch;
             int v[kRowBatch];
@@ -278,34 +288,20 @@ __global__ void __launch_bounds__(1024, 2) rows_kernel(DecodeArgs a) {
             const int pv = (lane == 0 && j0 > 0) ? __ldg(row + j0 - 1) : -1;
             int p = __shfl_up_sync(0xffffffffu, v[kRowBatch - 1], 1);
             if (lane == 0) p = pv;
-            int pg[kRowBatch];
 #pragma unroll
             for (int i = 0; i < kRowBatch; ++i) {
                 const int j = j0 + i;
-                pg[i] = -2;   // no cache row looked up
                 if (j < k_max) {
                     if (v[i] < 0) {
                         first_neg = min(first_neg, j);
                     } else if (v[i] >= n) {
                         report(a.status, SD_ERR_INDEX_OOB);
-                    } else {
-                        if (j > 0 && (p < 0 || p >= v[i])) report(a.status, SD_ERR_ORDER);
-                        pg[i] = __ldg(ptrow + (v[i] >> 4));
+                    } else if (j > 0 && (p < 0 || p >= v[i])) {
+                        report(a.status, SD_ERR_ORDER);
                     }
                 }
                 p = v[i];
             }
-            uint32_t ri[kRowBatch];
-#pragma unroll
-            for (int i = 0; i < kRowBatch; ++i) {
-                ri[i] = kNoRow;
-                if (pg[i] >= 0 && pg[i] < a.num_pages)
-                    ri[i] = ((uint32_t)pg[i] * kPageSize + (uint32_t)(v[i] & (kPageSize - 1))) * (uint32_t)a.Hkv + kvh;
-                else if (pg[i] != -2)
-                    report(a.status, SD_ERR_INDEX_OOB);
-            }
-            static_assert(kRowBatch == 4, "one 16-byte store per pass");
-            if (j0 < k_max) *reinterpret_cast<uint4*>(dst + j0) = make_uint4(ri[0], ri[1], ri[2], ri[3]);
         }
     }
     first_neg = __reduce_min_sync(0xffffffffu, first_neg);
@@ -335,68 +331,256 @@ __global__ void __launch_bounds__(1024, 2) rows_kernel(DecodeArgs a) {
 // ---------------------------------------------------------------------------------------------
 // sparse decode: sparse_decode_kernel
 // ---------------------------------------------------------------------------------------------
-// The warp's walk over its entries (all fields warp-uniform).
+// Shared memory of one decode warp: kSparseStages tiles of 16 gathered rows.  A tile holds four
+// 2 KB blocks -- K dims 0-63, K dims 64-127, V dims 0-63, V dims 64-127 -- each 16 rows of 128 B
+// with the 128-byte swizzle of the TMA copy (16-byte chunk c of row r stored at chunk c ^ (r & 7)),
+// so that ldmatrix reads eight rows of one chunk column without bank conflicts.
+constexpr int kHalfBlock = kTileRows * 128;                 // 2 KB: 16 rows x 64 dims
+constexpr int kGatherTile = 4 * kHalfBlock;                 // K and V, both halves
+struct SparseSmem {   // placed at a 1024-byte aligned address (swizzle atoms)
+    uint8_t kv[kSparseStages][kGatherTile];
+    uint64_t full[kSparseStages];           // TMA completion of each stage
+    int info[kSparseStages][4];             // rows | flags << 5 | valid-row mask << 16, row, segment slot, segments
+    uint32_t q[kSparseStages][kHeadDim / 2];   // q of the row a tile opens (bf16 pairs)
+};
+
+size_t sparse_decode_smem() { return sizeof(SparseSmem) + 1008; }   // + alignment slack (the base is 16-byte aligned)
+
+// The warp's walk over its entries.  Everything is warp-uniform; the per-row values are computed
+// once when the walk enters a row.
 struct RowWalker {
     int e, e_end;        // next entry (global order) and the end of this warp's share
     int epw;             // entries per warp
-    int r;               // row holding entry e
+    int r;               // row b * Hq + h holding entry e
     int rstart, rend;    // global entry range of row r
+    int next_len;        // length of row r + 1 (0 past the last row), loaded on entering row r
+    int seg;             // segment slot of this warp in row r | the row's segment count << 16
+    int pt_off;          // b * max_pages: row r's request in the page table
+    int kvh;             // KV head of row r
+    const int32_t* ix;   // idx of row r, indexed by global entry
     bool seg_new;        // the next tile opens a segment
+    int seq;             // tiles handed out so far
 };
 
-__device__ __forceinline__ TileDesc prefetch_row_tile(const DecodeArgs& a, RowWalker& w) {
+__device__ __forceinline__ void enter_row(const DecodeArgs& a, RowWalker& w, int r, int rstart, int len) {
+    const int R = a.B * a.Hq;
+    w.r = r;
+    w.rstart = rstart;
+    w.rend = rstart + len;
+    const int first_warp = rstart / w.epw;
+    w.seg = ((int)blockIdx.x - first_warp) | (((w.rend - 1) / w.epw - first_warp + 1) << 16);
+    const int b = r / a.Hq;
+    w.kvh = (r - b * a.Hq) / a.G;
+    w.pt_off = b * a.max_pages;
+    w.ix = a.idx + (long)r * a.k_max - rstart;
+    w.next_len = r + 1 < R ? __ldg(a.rlen + r + 1) : 0;
+    w.seg_new = true;
+}
+
+// One tile of the walk: warp-uniform fields, plus per lane (lanes < rows) the selected position v
+// and, one step later, its page-table entry.
+struct RowTile {
+    int hdr;            // rows | flags << 5 | stage << 8
+    int r, seg;         // row and segment (as in RowWalker)
+    int pt_off, kvh;
+    int v;              // this lane's position (lanes < rows)
+    int page;           // this lane's page-table entry (-1: not looked up)
+    uint2 q2;           // a tile that opens a row: this lane's 8 bytes of the row's q
+};
+
+// The next tile of the walk; issues the loads of its positions (first used two steps later).
+__device__ __forceinline__ RowTile next_row_tile(const DecodeArgs& a, RowWalker& w) {
     const int lane = threadIdx.x & 31;
-    TileDesc d = empty_tile();
-    if (w.e >= w.e_end) {
-        d.flags = kFlagEnd;
-        return d;
-    }
-    d.owner = w.r;
-    const int first_warp = w.rstart / w.epw;
-    d.seg_j = (int)blockIdx.x - first_warp;
-    d.nseg = (w.rend - 1) / w.epw - first_warp + 1;
-    if (w.seg_new) d.flags |= kFlagFirst;
-    w.seg_new = false;
+    RowTile d;
+    const int stage = w.seq++ & (kSparseStages - 1);
+    d.r = w.r;
+    d.seg = w.seg;
+    d.pt_off = w.pt_off;
+    d.kvh = w.kvh;
+    d.v = -1;
+    d.page = -1;
+    d.q2 = make_uint2(0u, 0u);
     const int rows = min(kTileRows, min(w.rend, w.e_end) - w.e);
-    if (rows <= 0) {   // not reached (row lengths and their sums come from one pass); ends the walk
+    if (rows <= 0) {   // the share is done (rows < 0 is not reached: lengths and sums come from one pass)
         w.e = w.e_end;
-        d.flags = kFlagEnd;
+        d.hdr = (kFlagEnd << 5) | (stage << 8);
         return d;
     }
-    if (lane < rows) {   // not examined until the tile is issued (one iteration later)
-        d.row_idx = __ldg(a.rowidx + (long)w.r * a.rstride + (w.e - w.rstart) + lane);
-        d.mask = 1u;
-    }
-    d.rows = rows;
+    int flags = w.seg_new ? kFlagFirst : 0;
+    w.seg_new = false;
+    if (lane < rows) d.v = __ldg(w.ix + w.e + lane);
     w.e += rows;
     if (w.e == w.rend || w.e == w.e_end) {
-        d.flags |= kFlagLast;
+        flags |= kFlagLast;
         if (w.e < w.e_end) {   // the next non-empty row (one exists: entries remain)
             const int R = a.B * a.Hq;
             int r = w.r + 1;
-            int len = __ldg(a.rlen + r);
+            int len = w.next_len;
             while (len == 0 && r + 1 < R) len = __ldg(a.rlen + (++r));
-            w.r = r;
-            w.rstart = w.rend;
-            w.rend = w.rstart + len;
-            w.seg_new = true;
+            enter_row(a, w, r, w.rend, len);
         }
     }
+    d.hdr = rows | (flags << 5) | (stage << 8);
     return d;
 }
 
-// Column 0 of the B operand is q[b][h]; the other columns are zero.
-__device__ __forceinline__ void load_q_row(const DecodeArgs& a, int r, Softmax<1>& st) {
-    const int lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
-    const uint32_t* qr = reinterpret_cast<const uint32_t*>(a.q + (long)r * kHeadDim);
+// Page-table lookup of the tile's positions (loaded two steps earlier), and the row's q when the
+// tile opens the row.  A position at or past N_b is reported by rows_kernel; here only positions
+// inside the page-table row (below max_pages * 16) are looked up.
+__device__ __forceinline__ void lookup_pages(const DecodeArgs& a, RowTile& d) {
+    const int lane = threadIdx.x & 31;
+    if (d.v >= 0 && d.v < a.n_cap) d.page = __ldg(a.page_table + d.pt_off + (d.v >> 4));
+    if ((d.hdr >> 5) & kFlagFirst) d.q2 = __ldg(reinterpret_cast<const uint2*>(a.q + (long)d.r * kHeadDim) + lane);
+}
+
+// 4-row gather of 128-byte half rows (2-D tensor [cache rows][128 dims], box {64, 1}) into shared
+// memory, completing on `bar`.
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const void* tmap, int x, int r0, int r1, int r2, int r3,
+                                            uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+        "%3, %4, %5, %6}], [%7];\n" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(bar)
+        : "memory");
+}
+
+// Maps the tile's positions to cache rows, records the tile in its stage and issues its gathers:
+// four four-row copies per 64-dim half of K and of V, issued by lane 0 (the copy takes its tensor
+// map and coordinates from one thread).  Rows past the tile's end or without a valid page repeat
+// the tile's first mapped row (an L2 hit) and are masked out: every row of the stage holds finite
+// data, since a masked row's zero weight still multiplies its V row.
+__device__ __forceinline__ void issue_row_tile(const DecodeArgs& a, SparseSmem& ws, uint32_t kv0, const RowTile& d,
+                                               const CUtensorMap* kmap, const CUtensorMap* vmap) {
+    const int lane = threadIdx.x & 31;
+    const int st = (d.hdr >> 8) & (kSparseStages - 1);
+    const int rows = d.hdr & 31;
+    bool ok = false;
+    uint32_t ri = 0;
+    if (d.v >= 0) {   // lanes < rows
+        if (d.page >= 0 && d.page < a.num_pages) {
+            ok = true;
+            ri = ((uint32_t)d.page * kPageSize + (uint32_t)(d.v & (kPageSize - 1))) * (uint32_t)a.Hkv + (uint32_t)d.kvh;
+        } else {
+            report(a.status, SD_ERR_INDEX_OOB);   // a page entry outside the cache, or a position at or past N_b
+        }
+    }
+    const uint32_t okm = __ballot_sync(0xffffffffu, ok);
+    if (lane == 0)
+        *reinterpret_cast<int4*>(ws.info[st]) = make_int4((d.hdr & 0xff) | (int)((okm & 0xffffu) << 16), d.r,
+                                                          d.seg & 0xffff, d.seg >> 16);
+    if ((d.hdr >> 5) & kFlagFirst) reinterpret_cast<uint2*>(ws.q[st])[lane] = d.q2;
+    if (rows == 0) return;
+    const uint32_t sub = okm ? __shfl_sync(0xffffffffu, ri, __ffs(okm) - 1) : 0u;   // every lane takes part
+    if (!ok) ri = sub;
+    const uint32_t bar = smem_addr(&ws.full[st]);
+    if (lane == 0) mbar_arrive_expect_tx(&ws.full[st], (uint32_t)kGatherTile);
+    const uint32_t dst = kv0 + (uint32_t)(st * kGatherTile);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        st.qb[0][j][0] = g == 0 ? __ldg(qr + 8 * j + c) : 0u;
-        st.qb[0][j][1] = g == 0 ? __ldg(qr + 8 * j + c + 4) : 0u;
+    for (int gq = 0; gq < kTileRows / 4; ++gq) {
+        const int q0 = __shfl_sync(0xffffffffu, (int)ri, 4 * gq + 0);
+        const int q1 = __shfl_sync(0xffffffffu, (int)ri, 4 * gq + 1);
+        const int q2 = __shfl_sync(0xffffffffu, (int)ri, 4 * gq + 2);
+        const int q3 = __shfl_sync(0xffffffffu, (int)ri, 4 * gq + 3);
+        if (lane == 0) {
+            const uint32_t o = (uint32_t)(gq * 4 * 128);
+            tma_gather4(dst + o, kmap, 0, q0, q1, q2, q3, bar);
+            tma_gather4(dst + kHalfBlock + o, kmap, 64, q0, q1, q2, q3, bar);
+            tma_gather4(dst + 2 * kHalfBlock + o, vmap, 0, q0, q1, q2, q3, bar);
+            tma_gather4(dst + 3 * kHalfBlock + o, vmap, 64, q0, q1, q2, q3, bar);
+        }
     }
 }
 
-// One warp: log-sum-exp merge of the nseg partials of row r (lane l owns dimensions 4l .. 4l+3).
+// Consumer state of one query head: the online softmax over its selected rows.  In the score MMA q
+// is column 0 of the B operand; in the P.V MMA column 0 carries the bf16 high part of the weights
+// and column 1 their bf16 residual, so the head's output is the sum of accumulator columns 0 and 1
+// (lanes with lane % 4 == 0 hold both).
+struct HeadState {
+    float m;            // running max of column 0 (log2 units; lanes % 4 == 0)
+    float l;            // partial sum of rows g, g + 8 (lanes % 4 == 0)
+    float acc[8][4];    // O^T fragments: dims 16 mt + g (+ 8) x columns 2 (lane % 4) (+ 1)
+    uint32_t qb[8][2];  // q as column 0 of the B operand
+};
+
+__device__ __forceinline__ void reset_head(HeadState& st) {
+    st.m = -INFINITY;
+    st.l = 0.f;
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) st.acc[mt][0] = st.acc[mt][1] = st.acc[mt][2] = st.acc[mt][3] = 0.f;
+}
+
+// q of the row from the stage (staged there when the tile was issued).
+__device__ __forceinline__ void load_q_head(const uint32_t* qr, HeadState& st) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        st.qb[j][0] = g == 0 ? qr[8 * j + c] : 0u;
+        st.qb[j][1] = g == 0 ? qr[8 * j + c + 4] : 0u;
+    }
+}
+
+// One tile: S = K_tile . q (8 MMAs), masked online softmax over the tile's valid rows, O^T += V_tile^T .
+// [p_hi, p_lo] (8 MMAs).  `koff` / `voff` are this lane's ldmatrix offsets (row and chunk, swizzled).
+__device__ __forceinline__ void compute_row_tile(const DecodeArgs& a, uint32_t tile, uint32_t valid,
+                                                 const uint32_t (&koff)[4], const uint32_t (&voff)[4],
+                                                 HeadState& st) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
+    float s[4] = {0.f, 0.f, 0.f, 0.f}, s2[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        uint32_t a0, a1, a2, a3;
+        ldmatrix_x4(tile + (uint32_t)((j >> 2) * kHalfBlock) + koff[j & 3], a0, a1, a2, a3);
+        if (j & 1) mma_bf16_16816(s2, a0, a1, a2, a3, st.qb[j][0], st.qb[j][1]);
+        else mma_bf16_16816(s, a0, a1, a2, a3, st.qb[j][0], st.qb[j][1]);
+    }
+    // column 0: rows g (s[0]) and g + 8 (s[2]) in lanes with c == 0
+    const float z0 = ((valid >> g) & 1u) ? (s[0] + s2[0]) * a.scale_log2 : -INFINITY;
+    const float z1 = ((valid >> (g + 8)) & 1u) ? (s[2] + s2[2]) * a.scale_log2 : -INFINITY;
+    float tm = fmaxf(z0, z1);
+    tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 4));
+    tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 8));
+    tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 16));
+    const float mo = st.m;
+    const float mn = fmaxf(mo, tm);
+    const float base = (mn == -INFINITY) ? 0.f : mn;
+    const float p0 = fast_exp2(z0 - base), p1 = fast_exp2(z1 - base);
+    const float al = (mo == mn || mo == -INFINITY) ? 1.f : fast_exp2(mo - mn);
+    st.l = st.l * al + p0 + p1;
+    st.m = mn;
+    if (__any_sync(0xffffffffu, al != 1.f)) {
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+            st.acc[mt][0] *= al;
+            st.acc[mt][1] *= al;
+            st.acc[mt][2] *= al;
+            st.acc[mt][3] *= al;
+        }
+    }
+    // B operand: lane (g', c') holds rows 2c', 2c'+1 (b0) and 2c'+8, 2c'+9 (b1) of column g';
+    // column 0 = bf16(p), column 1 = bf16(p - bf16(p)), the other columns zero.  Row i < 8 of the
+    // tile is p0 of lane 4 i, row i + 8 its p1.
+    const float pa0 = __shfl_sync(0xffffffffu, p0, 8 * c), pa1 = __shfl_sync(0xffffffffu, p0, 8 * c + 4);
+    const float pb0 = __shfl_sync(0xffffffffu, p1, 8 * c), pb1 = __shfl_sync(0xffffffffu, p1, 8 * c + 4);
+    const uint32_t h0 = pack_bf16x2(pa0, pa1), h1 = pack_bf16x2(pb0, pb1);
+    uint32_t b0 = 0u, b1 = 0u;
+    if (g == 0) {
+        b0 = h0;
+        b1 = h1;
+    } else if (g == 1) {
+        b0 = pack_bf16x2(pa0 - bf16_lo(h0), pa1 - bf16_hi(h0));
+        b1 = pack_bf16x2(pb0 - bf16_lo(h1), pb1 - bf16_hi(h1));
+    }
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+        uint32_t a0, a1, a2, a3;
+        ldmatrix_x4_trans(tile + (uint32_t)(2 * kHalfBlock + (mt >> 2) * kHalfBlock) + voff[mt & 3], a0, a1, a2, a3);
+        mma_bf16_16816(st.acc[mt], a0, a1, a2, a3, b0, b1);
+    }
+}
+
+// One warp: log-sum-exp merge of the nseg partials of row r (lane l owns dimensions 4l .. 4l+3),
+// kMergeBatch partial outputs per lane in flight together.
+constexpr int kMergeBatch = 8;
 __device__ __forceinline__ void merge_row(const DecodeArgs& a, int r, int nseg) {
     const int lane = threadIdx.x & 31;
     const float2* ml = a.ml + (long)r * a.jmax;
@@ -409,22 +593,24 @@ __device__ __forceinline__ void merge_row(const DecodeArgs& a, int r, int nseg) 
     }
     float L = 0.f;
     float4 o4 = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j0 = 0; j0 < nseg; j0 += 32) {
-        const float2 v = (j0 + lane < nseg) ? __ldcg(ml + j0 + lane) : make_float2(-INFINITY, 0.f);
-        const float wj = (v.x == -INFINITY) ? 0.f : exp2f(v.x - M);
-        float lw = wj * v.y;
+    const float4* src = reinterpret_cast<const float4*>(a.acc + (long)r * a.jmax * kHeadDim) + lane;
+    for (int j0 = 0; j0 < nseg; j0 += kMergeBatch) {
+        float4 x[kMergeBatch];
+        float2 v[kMergeBatch];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) lw += __shfl_xor_sync(0xffffffffu, lw, o);
-        L += lw;
-        const int cnt = min(32, nseg - j0);
-        const float4* src = reinterpret_cast<const float4*>(a.acc + ((long)r * a.jmax + j0) * kHeadDim) + lane;
-        for (int jj = 0; jj < cnt; ++jj) {
-            const float ww = __shfl_sync(0xffffffffu, wj, jj);
-            const float4 x = __ldcg(src + (long)jj * (kHeadDim / 4));
-            o4.x += ww * x.x;
-            o4.y += ww * x.y;
-            o4.z += ww * x.z;
-            o4.w += ww * x.w;
+        for (int i = 0; i < kMergeBatch; ++i) {   // clamped (in-range) loads, all in flight together
+            const int j = min(j0 + i, nseg - 1);
+            x[i] = __ldcg(src + (long)j * (kHeadDim / 4));
+            v[i] = __ldcg(ml + j);
+        }
+#pragma unroll
+        for (int i = 0; i < kMergeBatch; ++i) {
+            const float wj = (j0 + i >= nseg || v[i].x == -INFINITY) ? 0.f : exp2f(v[i].x - M);
+            L += wj * v[i].y;
+            o4.x += wj * x[i].x;
+            o4.y += wj * x[i].y;
+            o4.z += wj * x[i].z;
+            o4.w += wj * x[i].w;
         }
     }
     const float inv = L > 0.f ? 1.f / L : 0.f;
@@ -432,10 +618,10 @@ __device__ __forceinline__ void merge_row(const DecodeArgs& a, int r, int nseg) 
         make_float4(o4.x * inv, o4.y * inv, o4.z * inv, o4.w * inv);
 }
 
-// End of this warp's segment of row r (column 0 of the state).
-__device__ __forceinline__ void finish_row_segment(const DecodeArgs& a, int r, int j, int nseg, Softmax<1>& st) {
+// End of this warp's segment of row r.
+__device__ __forceinline__ void finish_row_segment(const DecodeArgs& a, int r, int j, int nseg, const HeadState& st) {
     const int lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
-    float l = st.l[0][0];
+    float l = st.l;
     l += __shfl_xor_sync(0xffffffffu, l, 4);
     l += __shfl_xor_sync(0xffffffffu, l, 8);
     l += __shfl_xor_sync(0xffffffffu, l, 16);
@@ -445,20 +631,20 @@ __device__ __forceinline__ void finish_row_segment(const DecodeArgs& a, int r, i
             float* dst = a.out + (long)r * kHeadDim;
 #pragma unroll
             for (int mt = 0; mt < 8; ++mt) {
-                dst[16 * mt + g] = st.acc[0][mt][0] * inv;
-                dst[16 * mt + g + 8] = st.acc[0][mt][2] * inv;
+                dst[16 * mt + g] = (st.acc[mt][0] + st.acc[mt][1]) * inv;
+                dst[16 * mt + g + 8] = (st.acc[mt][2] + st.acc[mt][3]) * inv;
             }
         }
         return;
     }
     const long slot = (long)r * a.jmax + j;
-    if (lane == 0) a.ml[slot] = make_float2(st.m[0][0], l);
+    if (lane == 0) a.ml[slot] = make_float2(st.m, l);
     if (c == 0) {
         float* dst = a.acc + slot * kHeadDim;
 #pragma unroll
         for (int mt = 0; mt < 8; ++mt) {
-            dst[16 * mt + g] = st.acc[0][mt][0];
-            dst[16 * mt + g + 8] = st.acc[0][mt][2];
+            dst[16 * mt + g] = st.acc[mt][0] + st.acc[mt][1];
+            dst[16 * mt + g + 8] = st.acc[mt][2] + st.acc[mt][3];
         }
     }
     __threadfence();   // this partial is visible before the arrival is counted
@@ -471,24 +657,28 @@ __device__ __forceinline__ void finish_row_segment(const DecodeArgs& a, int r, i
     merge_row(a, r, nseg);
 }
 
-__global__ void __launch_bounds__(32) sparse_decode_kernel(DecodeArgs a) {
-    extern __shared__ __align__(128) uint8_t smem[];
-    DecodeSmem& ws = *reinterpret_cast<DecodeSmem*>(smem);
+__global__ void __launch_bounds__(32) sparse_decode_kernel(DecodeArgs a, const __grid_constant__ CUtensorMap kmap,
+                                                           const __grid_constant__ CUtensorMap vmap) {
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    SparseSmem& ws = *reinterpret_cast<SparseSmem*>(
+        smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u));   // 1024-byte aligned (swizzle atoms)
+    const int lane = threadIdx.x & 31;
+    if (lane == 0) {
+#pragma unroll
+        for (int s = 0; s < kSparseStages; ++s) mbar_init(&ws.full[s], 1);
+        mbar_fence_init();
+    }
+    __syncwarp();
     pdl_enter();
 
-    const int lane = threadIdx.x & 31;
     const int R = a.B * a.Hq;
-    // E = all entries: the length sums of the rows_kernel CTAs, kPrologue per lane in flight together
+    // E = all entries: the length sums of the rows_kernel CTAs, each lane summing kPrologue
+    // consecutive ones per round
     int E = 0;
     for (int base = 0; base < a.nb; base += 32 * kPrologue) {
-        int v[kPrologue];
+        const int k0 = base + kPrologue * lane;
 #pragma unroll
-        for (int i = 0; i < kPrologue; ++i) {
-            const int k = base + 32 * i + lane;
-            v[i] = k < a.nb ? __ldg(a.bsum + k) : 0;
-        }
-#pragma unroll
-        for (int i = 0; i < kPrologue; ++i) E += v[i];
+        for (int i = 0; i < kPrologue; ++i) E += k0 + i < a.nb ? __ldg(a.bsum + k0 + i) : 0;
     }
     E = __reduce_add_sync(0xffffffffu, E);
     if (E == 0) return;
@@ -498,36 +688,43 @@ __global__ void __launch_bounds__(32) sparse_decode_kernel(DecodeArgs a) {
     if (e0 >= E) return;
     w.e = (int)e0;
     w.e_end = (int)min((long)E, e0 + w.epw);
-    // the rows_kernel CTA whose rows hold entry w.e (prefix over the same sums, now in L1), then the row
+    // the rows_kernel CTA whose rows hold entry w.e: one scan of the lanes' sums per round (the
+    // sums are in L1 now), then the lane that holds it walks its kPrologue sums
     int blk = -1, blk0 = 0, blen = 0;
     {
         int acc = 0;
         for (int base = 0; base < a.nb && blk < 0; base += 32 * kPrologue) {
-            int v[kPrologue];
+            const int k0 = base + kPrologue * lane;
+            int v[kPrologue], sum = 0;
 #pragma unroll
             for (int i = 0; i < kPrologue; ++i) {
-                const int k = base + 32 * i + lane;
-                v[i] = k < a.nb ? __ldg(a.bsum + k) : 0;
+                v[i] = k0 + i < a.nb ? __ldg(a.bsum + k0 + i) : 0;
+                sum += v[i];
             }
+            const int incl = warp_inclusive_scan(sum);
+            const uint32_t hit = __ballot_sync(0xffffffffu, acc + incl > w.e);
+            if (hit != 0u) {
+                const int l = __ffs(hit) - 1;
+                int c = acc + incl - sum, kb = -1, kb0 = 0, kl = 0;   // lane l: its sums in order
 #pragma unroll
-            for (int i = 0; i < kPrologue; ++i) {
-                const int incl = warp_inclusive_scan(v[i]);
-                const uint32_t hit = __ballot_sync(0xffffffffu, acc + incl > w.e);
-                if (blk < 0 && hit != 0u) {
-                    const int l = __ffs(hit) - 1;
-                    blk = base + 32 * i + l;
-                    blk0 = acc + __shfl_sync(0xffffffffu, incl - v[i], l);
-                    blen = __shfl_sync(0xffffffffu, v[i], l);
+                for (int i = 0; i < kPrologue; ++i) {
+                    if (kb < 0 && c + v[i] > w.e) {
+                        kb = k0 + i;
+                        kb0 = c;
+                        kl = v[i];
+                    }
+                    c += v[i];
                 }
-                acc += __shfl_sync(0xffffffffu, incl, 31);
+                blk = __shfl_sync(0xffffffffu, kb, l);
+                blk0 = __shfl_sync(0xffffffffu, kb0, l);
+                blen = __shfl_sync(0xffffffffu, kl, l);
             }
+            acc += __shfl_sync(0xffffffffu, incl, 31);
         }
     }
     if (blk < 0) return;   // not reached: w.e < E
     if (a.rpc == 1) {      // one row per CTA of the row pass
-        w.r = blk;
-        w.rstart = blk0;
-        w.rend = blk0 + blen;
+        enter_row(a, w, blk, blk0, blen);
     } else {
         const int r0 = blk * a.rpc;
         const int v = (lane < a.rpc && r0 + lane < R) ? __ldg(a.rlen + r0 + lane) : 0;
@@ -535,39 +732,73 @@ __global__ void __launch_bounds__(32) sparse_decode_kernel(DecodeArgs a) {
         const uint32_t hit = __ballot_sync(0xffffffffu, blk0 + incl > w.e);
         if (hit == 0u) return;   // not reached: the CTA's rows hold entry w.e
         const int l = __ffs(hit) - 1;
-        w.r = r0 + l;
-        w.rstart = blk0 + __shfl_sync(0xffffffffu, incl - v, l);
-        w.rend = w.rstart + __shfl_sync(0xffffffffu, v, l);
+        enter_row(a, w, r0 + l, blk0 + __shfl_sync(0xffffffffu, incl - v, l), __shfl_sync(0xffffffffu, v, l));
     }
-    w.seg_new = true;
+    w.seq = 0;
 
-    Softmax<1> st;
-    reset_state(st);
-    TileDesc next = prefetch_row_tile(a, w);
+    // this lane's ldmatrix offsets inside a 2 KB half block: K (A operand, rows 8 (lane>>3 & 1) +
+    // (lane & 7), chunk 2 (j & 3) + (lane >> 4)) and V (A operand transposed, rows 8 (lane >> 4) +
+    // (lane & 7), chunk 2 (mt & 3) + (lane >> 3 & 1)), each chunk swizzled by the row's low 3 bits
+    uint32_t koff[4], voff[4];
+    {
+        const int rk = (((lane >> 3) & 1) << 3) + (lane & 7), rv = ((lane >> 4) << 3) + (lane & 7);
 #pragma unroll
-    for (int s = 0; s < kStages - 1; ++s) {
-        issue_tile(a, ws, s, next);
-        next = prefetch_row_tile(a, w);
-    }
-    for (int t = 0;; ++t) {
-        const int stage = t % kStages;
-        // the stage of tile t-1 is free: issue tile t+kStages-1 before waiting for tile t
-        issue_tile(a, ws, (t + kStages - 1) % kStages, next);
-        next = prefetch_row_tile(a, w);
-        cp_async_wait<kStages - 1>();
-        __syncwarp();
-        const int rows = ws.info[stage][0], flags = ws.info[stage][1];
-        if (flags & kFlagEnd) break;
-        const int r = ws.info[stage][2], j = ws.info[stage][3], nseg = ws.info[stage][4];
-        if (flags & kFlagFirst) load_q_row(a, r, st);
-        if (rows > 0) compute_tile(a, ws, stage, st);
-        if (flags & kFlagLast) {
-            finish_row_segment(a, r, j, nseg, st);
-            reset_state(st);
+        for (int jj = 0; jj < 4; ++jj) {
+            koff[jj] = (uint32_t)(rk * 128 + (((2 * jj + (lane >> 4)) ^ (lane & 7)) << 4));
+            voff[jj] = (uint32_t)(rv * 128 + (((2 * jj + ((lane >> 3) & 1)) ^ (lane & 7)) << 4));
         }
-        __syncwarp();
     }
-    cp_async_wait<0>();
+    const uint32_t kv0 = smem_addr(ws.kv);
+
+    // Software pipeline over tiles, so that no load but the gather itself is waited for: while tile
+    // t is consumed, tile t + 1 is gathered (its pages were looked up a step earlier), the pages of
+    // tile t + 2 are looked up (its positions were loaded two steps earlier) and the positions of
+    // tile t + 4 are loaded.
+    static_assert(kSparseStages == 2, "the pipeline below gathers one tile ahead");
+    // (Each page lookup follows the rotation of the records, so that no record is copied while a
+    // load into it is in flight: such a register copy would wait for the load.)
+    RowTile dA = next_row_tile(a, w), dB = next_row_tile(a, w), dC = next_row_tile(a, w);
+    lookup_pages(a, dA);
+    issue_row_tile(a, ws, kv0, dA, &kmap, &vmap);   // tile 0
+    dA = dB;
+    dB = dC;
+    dC = next_row_tile(a, w);
+    lookup_pages(a, dA);
+    HeadState st;
+    reset_head(st);
+    bool ok = true;
+    int t = 0;
+    for (;; ++t) {
+        const int stage = t & (kSparseStages - 1);
+        issue_row_tile(a, ws, kv0, dA, &kmap, &vmap);   // into the stage tile t - 1 used
+        dA = dB;
+        dB = dC;
+        dC = next_row_tile(a, w);
+        lookup_pages(a, dA);
+        __syncwarp();
+        const int4 info = *reinterpret_cast<const int4*>(ws.info[stage]);
+        const int flags = (info.x >> 5) & 7;
+        if (flags & kFlagEnd) break;
+        if (flags & kFlagFirst) load_q_head(ws.q[stage], st);
+        ok = mbar_wait(&ws.full[stage], (uint32_t)((t / kSparseStages) & 1));
+        ok = __all_sync(0xffffffffu, ok);   // warp-uniform before the collective ops below
+        if (!ok) break;
+        compute_row_tile(a, kv0 + (uint32_t)(stage * kGatherTile), (uint32_t)info.x >> 16, koff, voff, st);
+        if (flags & kFlagLast) {
+            finish_row_segment(a, info.y, info.z, info.w, st);
+            reset_head(st);
+        }
+        __syncwarp();   // every lane has read the stage before it is refilled
+    }
+    if (!ok) {
+        // A copy never completed: record it, wait (bounded) for this warp's copies still in
+        // flight, and return; the rows this warp held are left unwritten.
+        if (lane == 0) report(a.status, SD_ERR_TIMEOUT);
+        for (int u = t; u < t + kSparseStages; ++u) {
+            const int hdr = ws.info[u % kSparseStages][0];
+            if ((hdr & 31) > 0) mbar_wait(&ws.full[u % kSparseStages], (uint32_t)((u / kSparseStages) & 1));
+        }
+    }
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -920,14 +1151,80 @@ static cudaError_t occupancy_of(K kernel, int* ctas) {
 }
 
 cudaError_t decode_occupancy(bool dense, int G, int* ctas_per_sm) {
-    if (!dense) return occupancy_of(sparse_decode_kernel, ctas_per_sm);
+    if (!dense) {
+        const size_t smem = sparse_decode_smem();
+        cudaError_t e = cudaFuncSetAttribute(sparse_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, sparse_decode_kernel, 32, smem);
+    }
     return G <= 8 ? occupancy_of(dense_decode_kernel<1>, ctas_per_sm) : occupancy_of(dense_decode_kernel<2>, ctas_per_sm);
 }
 
-cudaError_t launch_sparse(const DecodeArgs& a, cudaStream_t stream) {
-    cudaError_t e = launch_pdl(rows_kernel, dim3(a.nb), dim3(a.tpr * a.rpc), 0, stream, a);
+namespace {
+
+// The K and V caches as 2-D tensors [num_pages * 16 * Hkv cache rows][128 dims] for the row
+// gathers: box {64 dims, 1 row}, 128-byte swizzle.  Encoded on the host through the driver entry
+// point, and kept for the last (device, K, V, rows).
+struct RowMapCache {
+    std::mutex mu;
+    PFN_cuTensorMapEncodeTiled encode = nullptr;
+    int dev = -1;
+    const void* K = nullptr;
+    const void* V = nullptr;
+    long rows = 0;
+    CUtensorMap kmap, vmap;
+};
+RowMapCache g_rowmap;
+
+CUresult encode_rows(PFN_cuTensorMapEncodeTiled encode, CUtensorMap* m, const void* base, long rows) {
+    const cuuint64_t dims[2] = {(cuuint64_t)kHeadDim, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)kRowBytes};
+    const cuuint32_t box[2] = {64, 1};
+    const cuuint32_t estr[2] = {1, 1};
+    return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+cudaError_t row_tensor_maps(const DecodeArgs& a, CUtensorMap* kmap, CUtensorMap* vmap) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(sparse_decode_kernel, dim3(a.total_warps), dim3(32), decode_smem(), stream, a);
+    const long rows = (long)a.num_pages * kPageSize * a.Hkv;
+    std::lock_guard<std::mutex> lock(g_rowmap.mu);
+    if (g_rowmap.encode == nullptr) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+        if (e != cudaSuccess) return e;
+        if (q != cudaDriverEntryPointSuccess || fn == nullptr) return cudaErrorNotSupported;
+        g_rowmap.encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled>(fn);
+    }
+    if (g_rowmap.dev != dev || g_rowmap.K != a.K || g_rowmap.V != a.V || g_rowmap.rows != rows) {
+        if (encode_rows(g_rowmap.encode, &g_rowmap.kmap, a.K, rows) != CUDA_SUCCESS ||
+            encode_rows(g_rowmap.encode, &g_rowmap.vmap, a.V, rows) != CUDA_SUCCESS) {
+            g_rowmap.dev = -1;
+            return cudaErrorInvalidValue;
+        }
+        g_rowmap.dev = dev;
+        g_rowmap.K = a.K;
+        g_rowmap.V = a.V;
+        g_rowmap.rows = rows;
+    }
+    *kmap = g_rowmap.kmap;
+    *vmap = g_rowmap.vmap;
+    return cudaSuccess;
+}
+
+}  // namespace
+
+cudaError_t launch_sparse(const DecodeArgs& a, cudaStream_t stream) {
+    CUtensorMap kmap, vmap;
+    cudaError_t e = row_tensor_maps(a, &kmap, &vmap);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(rows_kernel, dim3(a.nb), dim3(a.tpr * a.rpc), 0, stream, a);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(sparse_decode_kernel, dim3(a.total_warps), dim3(32), sparse_decode_smem(), stream, a, kmap, vmap);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 

@@ -73,12 +73,12 @@ def test_workspace_sizes(lib):
     scores = rows * 8192 * 16 * 4                          # fp32 candidate streams, B*Hq*n_cap
     small = rows * 8192 * 8 + rows * 4 + 3 * 8             # (head, page) records, thresholds, pointers
     assert scores + small <= topk <= scores + small + 4 * 256
-    # sparse decode: 64 segment partials per (b, h) row (fp32 output + max and sum), the cache row of
-    # every idx entry (rows k_max rounded up to 4 entries apart), and per row its length and arrival
-    # counter; then one length sum per CTA of the row pass (1 row per CTA at k_max 2621)
+    # sparse decode: 64 segment partials per (b, h) row (fp32 output + max and sum), per row its
+    # length and arrival counter, then one length sum per CTA of the row pass (1 row per CTA at
+    # k_max 2621)
     sparse = sdb.sd_workspace_size(s, sdb.SD_OP_SPARSE)
-    need = rows * 64 * (128 * 4 + 8) + rows * 2624 * 4 + rows * 4 * 2 + rows * 4
-    assert need <= sparse <= need + 6 * 256
+    need = rows * 64 * (128 * 4 + 8) + rows * 4 * 2 + rows * 4
+    assert need <= sparse <= need + 5 * 256
     # dense decode: min(N, 1280) + 1 segment partials per (b, h) and one row count per 16384 positions
     # of every (b, KV head) group
     dense = sdb.sd_workspace_size(s, sdb.SD_OP_DENSE)
