@@ -68,8 +68,12 @@ def _configure(lib):
     lib.oracle_dense.argtypes = [I] * 7 + [P, P, P, P, P, P]
     lib.oracle_quest_scores.argtypes = [I] * 7 + [P, P, P, P, I, I, P]
     lib.oracle_quest_topk.argtypes = [I] * 8 + [P, P, P, P, P, P]
+    lib.oracle_attend_parts.argtypes = [I] * 8 + [P, P, P, P, P, P, P, P]
+    lib.oracle_stochastic_topk.argtypes = [I] * 8 + [P, P, P, P, P, P, ctypes.c_uint64, ctypes.c_uint32, P]
+    lib.oracle_splitmix64.argtypes = [ctypes.c_uint64]
+    lib.oracle_splitmix64.restype = ctypes.c_uint64
     for f in (lib.oracle_scores, lib.oracle_topk, lib.oracle_attend, lib.oracle_dense, lib.oracle_quest_scores,
-              lib.oracle_quest_topk):
+              lib.oracle_quest_topk, lib.oracle_attend_parts, lib.oracle_stochastic_topk):
         f.restype = ctypes.c_int
     lib.oracle_num_threads.restype = ctypes.c_int
     return lib
@@ -193,3 +197,41 @@ def quest_topk(shape: dict, q, K, page_table, lens, k, k_max: int | None = None)
     _check(_load().oracle_quest_topk(B, Hq, Hkv, d, P, max_pages, num_pages, k_max, _p(qa), _p(Ka), _p(pt),
                                      _p(ln), _p(ka), _p(idx)), "quest_topk")
     return idx
+
+
+SAMPLED_FLAG = 1 << 30   # idx entry of a row drawn by the stochastic selection (position in the low 30 bits)
+
+
+def splitmix64(x: int) -> int:
+    """One output of the SplitMix64 generator from state x (the oracle's sampling hash)."""
+    return int(_load().oracle_splitmix64(ctypes.c_uint64(x & 0xFFFFFFFFFFFFFFFF)))
+
+
+def stochastic_topk(shape: dict, q, K, page_table, lens, k_det, k_samp, seed: int, step: int,
+                    k_max: int | None = None) -> np.ndarray:
+    """Stochastic selection: exact top-k_det plus min(k_samp, |rest|) rows drawn uniformly without
+    replacement from the rest (smallest sampling keys), ascending, sampled rows flagged."""
+    B, Hq, Hkv, d, P, max_pages = _dims(shape)
+    k_max = int(shape["k_max"] if k_max is None else k_max)
+    qa, Ka, pt, ln, kd, ks = _u16(q), _u16(K), _i32(page_table), _i32(lens), _i32(k_det), _i32(k_samp)
+    num_pages = Ka.size // (P * Hkv * d)
+    idx = np.full((B, Hq, max(k_max, 0)), -1, dtype=np.int32)
+    _check(_load().oracle_stochastic_topk(B, Hq, Hkv, d, P, max_pages, num_pages, k_max, _p(qa), _p(Ka), _p(pt),
+                                          _p(ln), _p(kd), _p(ks), ctypes.c_uint64(seed & 0xFFFFFFFFFFFFFFFF),
+                                          ctypes.c_uint32(step & 0xFFFFFFFF), _p(idx)), "stochastic_topk")
+    return idx
+
+
+def attend_parts(shape: dict, q, K, V, page_table, lens, idx):
+    """Unnormalised numerator [B, Hq, d] and denominator [B, Hq] of attend (exps relative to 0)."""
+    B, Hq, Hkv, d, P, max_pages = _dims(shape)
+    qa, Ka, Va, pt, ln = _u16(q), _u16(K), _u16(V), _i32(page_table), _i32(lens)
+    ix = _i32(idx)
+    k_max = ix.shape[-1]
+    num_pages = Ka.size // (P * Hkv * d)
+    num = np.zeros((B, Hq, d), dtype=np.float64)
+    den = np.zeros((B, Hq), dtype=np.float64)
+    _check(_load().oracle_attend_parts(B, Hq, Hkv, d, P, max_pages, num_pages, k_max, _p(qa), _p(Ka), _p(Va),
+                                       _p(pt), _p(ln), _p(ix), _p(num), _p(den)), "attend_parts")
+    return num, den
+

@@ -29,6 +29,20 @@
  *              r_j = sum_d max(q_d * min_d, q_d * max_d).  Budget: ceil(k_b / P) pages (the
  *              current page plus the best others, ties to the lower page); the selection is
  *              every position < N_b of the kept pages, ascending.
+ *   stochastic the stochastic index selection the pages evaluate (vAttention: "Technische
+ *              Zusammenfassung", sec. 2 "Stochastische Indexierung" and sec. 3A "Stochastisch vs.
+ *              Deterministisch"), which they name but do not spell out.  The reading here: per
+ *              (b, h) the exact top-k_det rows S_d (as in select), plus m = min(k_samp, |R|) rows
+ *              S_s drawn uniformly without replacement from the rest R = [0, N_b) \ S_d; each
+ *              sampled row stands for |R| / m rows, i.e. its exp(z) is multiplied by w = |R| / m
+ *              in both the numerator and the denominator of the softmax (an inverse-inclusion-
+ *              probability estimate of the sums over R).  The draw: every p in R gets the key
+ *              u(p) = top 32 bits of SM(SM(SM(seed + step) + r) + p), r = b * Hq + h, where
+ *              SM(x) is one output of the SplitMix64 generator from state x (Steele, Lea and
+ *              Flood, "Fast splittable pseudorandom number generators", 2014); S_s = the m
+ *              positions with the smallest (u, p).  In idx a sampled row carries bit 30
+ *              (SAMPLED_FLAG) on its position; attend reads w back from the row as
+ *              (N_b - #unflagged) / #flagged.
  *
  * Data layout read here (the paged KV cache the pages describe as a paged-KV backend,
  * "Inference-time context sparsity", sec. 1, "sparsity is usable for systems gains"):
@@ -51,6 +65,9 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+
+#define SAMPLED_FLAG 0x40000000   /* idx entry: a row drawn by the stochastic selection */
+#define POS_MASK 0x3fffffff
 
 /* bf16 -> double is exact: a bf16 is the top half of an IEEE binary32. */
 static double bf16_to_double(uint16_t bits) {
@@ -174,24 +191,30 @@ int oracle_topk(int B, int Hq, int Hkv, int d, int P, int max_pages, int num_pag
     return rc_all;
 }
 
-/* Softmax attention of one (b, h) over the listed positions (order irrelevant):
- * z_i = s_i / sqrt(d), w_i = exp(z_i - max z), out = sum w_i V_i / sum w_i.
- * An empty list gives out = 0. */
-static int attend_one(const oshape* s, const uint16_t* q, const uint16_t* K, const uint16_t* V,
-                      const int32_t* page_table, int b, int h, int n, const int32_t* sel, int nsel,
-                      double* out) {
+/* The two sums of softmax attention of one (b, h) over the listed rows (order irrelevant), each
+ * exp taken relative to zref:  z_i = s_i / sqrt(d),  e_i = c_i exp(z_i - zref),
+ * num = sum e_i V_i (d doubles),  den = sum e_i,  with c_i = 1 for a plain entry and
+ * c_i = w = (N_b - #plain) / #sampled for an entry that carries SAMPLED_FLAG.
+ * zref < -1e300 asks for zref = max z_i (the numerically safe choice). */
+static int attention_sums(const oshape* s, const uint16_t* q, const uint16_t* K, const uint16_t* V,
+                          const int32_t* page_table, int b, int h, int n, const int32_t* sel, int nsel,
+                          double zref, double* num, double* den) {
     int G = s->Hq / s->Hkv;
     int kvh = h / G;
     const uint16_t* qh = q + ((long)b * s->Hq + h) * s->d;
-    for (int j = 0; j < s->d; ++j) out[j] = 0.0;
+    for (int j = 0; j < s->d; ++j) num[j] = 0.0;
+    *den = 0.0;
     if (nsel == 0) return 0;
+    int nsamp = 0;
+    for (int t = 0; t < nsel; ++t) nsamp += (sel[t] & SAMPLED_FLAG) != 0;
+    double w = nsamp > 0 ? (double)(n - (nsel - nsamp)) / (double)nsamp : 1.0;
     double* z = (double*)malloc(sizeof(double) * (size_t)nsel);
     if (!z) return -4;
     double scale = 1.0 / sqrt((double)s->d);
     double zmax = -INFINITY;
     for (int t = 0; t < nsel; ++t) {
-        int32_t p = sel[t];
-        if (p < 0 || p >= n) { free(z); return -2; }
+        int32_t p = sel[t] & POS_MASK;
+        if (p >= n) { free(z); return -2; }
         const uint16_t* krow = cache_row(s, K, page_table, b, kvh, p);
         if (!krow) { free(z); return -2; }
         double acc = 0.0;
@@ -199,21 +222,31 @@ static int attend_one(const oshape* s, const uint16_t* q, const uint16_t* K, con
         z[t] = acc * scale;
         if (z[t] > zmax) zmax = z[t];
     }
-    double denom = 0.0;
+    if (zref < -1e300) zref = zmax;
     for (int t = 0; t < nsel; ++t) {
-        double w = exp(z[t] - zmax);
-        const uint16_t* vrow = cache_row(s, V, page_table, b, kvh, sel[t]);
+        double e = exp(z[t] - zref) * ((sel[t] & SAMPLED_FLAG) ? w : 1.0);
+        const uint16_t* vrow = cache_row(s, V, page_table, b, kvh, sel[t] & POS_MASK);
         if (!vrow) { free(z); return -2; }
-        denom += w;
-        for (int j = 0; j < s->d; ++j) out[j] += w * bf16_to_double(vrow[j]);
+        *den += e;
+        for (int j = 0; j < s->d; ++j) num[j] += e * bf16_to_double(vrow[j]);
     }
-    for (int j = 0; j < s->d; ++j) out[j] /= denom;
     free(z);
     return 0;
 }
 
-/* Attention over the rows each (b, h) lists in idx (entries < 0 are padding and are skipped).
- * out is double [B][Hq][d]. */
+/* Softmax attention of one (b, h) over the listed rows: out = num / den (an empty list gives 0). */
+static int attend_one(const oshape* s, const uint16_t* q, const uint16_t* K, const uint16_t* V,
+                      const int32_t* page_table, int b, int h, int n, const int32_t* sel, int nsel,
+                      double* out) {
+    double den = 0.0;
+    int rc = attention_sums(s, q, K, V, page_table, b, h, n, sel, nsel, -INFINITY, out, &den);
+    if (rc != 0 || nsel == 0) return rc;
+    for (int j = 0; j < s->d; ++j) out[j] /= den;
+    return 0;
+}
+
+/* Attention over the rows each (b, h) lists in idx (entries < 0 are padding and are skipped;
+ * entries with SAMPLED_FLAG are weighted as described at the top).  out is double [B][Hq][d]. */
 int oracle_attend(int B, int Hq, int Hkv, int d, int P, int max_pages, int num_pages, int k_max,
                   const uint16_t* q, const uint16_t* K, const uint16_t* V, const int32_t* page_table,
                   const int32_t* lens, const int32_t* idx, double* out) {
@@ -260,6 +293,121 @@ int oracle_dense(int B, int Hq, int Hkv, int d, int P, int max_pages, int num_pa
             rc = attend_one(&s, q, K, V, page_table, b, h, n, sel, n, out + bh * (long)d);
         }
         free(sel);
+        if (rc < rc_all) rc_all = rc;
+    }
+    return rc_all;
+}
+
+/* The unnormalised sums of attend, every exp taken relative to 0 (so that sums from different
+ * row lists are comparable): num double [B][Hq][d], den double [B][Hq]. */
+int oracle_attend_parts(int B, int Hq, int Hkv, int d, int P, int max_pages, int num_pages, int k_max,
+                        const uint16_t* q, const uint16_t* K, const uint16_t* V, const int32_t* page_table,
+                        const int32_t* lens, const int32_t* idx, double* num, double* den) {
+    oshape s = {B, Hq, Hkv, d, P, max_pages, k_max, num_pages};
+    if (check_shape(&s)) return -1;
+    for (int b = 0; b < B; ++b)
+        if (req_len(&s, lens, b) < 0) return -1;
+    int rc_all = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(min : rc_all)
+    for (long bh = 0; bh < (long)B * Hq; ++bh) {
+        int b = (int)(bh / Hq), h = (int)(bh % Hq);
+        const int32_t* row = idx + bh * (long)k_max;
+        int32_t* sel = (int32_t*)malloc(sizeof(int32_t) * (size_t)(k_max > 0 ? k_max : 1));
+        int nsel = 0;
+        int rc = sel ? 0 : -4;
+        if (sel) {
+            for (int t = 0; t < k_max; ++t)
+                if (row[t] >= 0) sel[nsel++] = row[t];
+            rc = attention_sums(&s, q, K, V, page_table, b, h, lens[b], sel, nsel, 0.0, num + bh * (long)d, den + bh);
+        }
+        free(sel);
+        if (rc < rc_all) rc_all = rc;
+    }
+    return rc_all;
+}
+
+/* One output of the SplitMix64 generator whose state is x before the step: the state advances by
+ * the golden-ratio increment 0x9E3779B97F4A7C15 and is then mixed (Steele, Lea and Flood 2014). */
+static uint64_t splitmix64(uint64_t x) {
+    uint64_t z = x + 0x9E3779B97F4A7C15ull;
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    return z ^ (z >> 31);
+}
+
+uint64_t oracle_splitmix64(uint64_t x) { return splitmix64(x); }
+
+/* Sampling key of position p in row r: the top 32 bits of SM(SM(SM(seed + step) + r) + p). */
+static uint32_t sample_key(uint64_t seed, uint32_t step, long r, long p) {
+    uint64_t c = splitmix64(splitmix64(splitmix64(seed + (uint64_t)step) + (uint64_t)r) + (uint64_t)p);
+    return (uint32_t)(c >> 32);
+}
+
+typedef struct { uint32_t key; int32_t pos; } keyed;
+
+static int by_key_then_pos(const void* a, const void* b) {
+    const keyed* x = (const keyed*)a;
+    const keyed* y = (const keyed*)b;
+    if (x->key != y->key) return (x->key < y->key) ? -1 : 1;
+    return (x->pos < y->pos) ? -1 : (x->pos > y->pos);
+}
+
+/* Stochastic selection of one (b, h) (see the top): S_d = exact top-k_det, S_s = the min(k_samp, |R|)
+ * positions of R = [0, N_b) \ S_d with the smallest sampling keys; both ascending together in
+ * idx_row, sampled ones with SAMPLED_FLAG, then -1. */
+static int stochastic_one(const oshape* s, const uint16_t* q, const uint16_t* K, const int32_t* page_table,
+                          int b, int h, int n, int kdet, int ksamp, uint64_t seed, uint32_t step, int32_t* idx_row) {
+    int rc = topk_one(s, q, K, page_table, b, h, n, kdet, idx_row);
+    if (rc != 0 || n <= 0) return rc;
+    int ndet = 0;   /* the rows top-k returned */
+    while (ndet < s->k_max && idx_row[ndet] >= 0) ++ndet;
+    long nrest = (long)n - ndet;
+    long m = ksamp < nrest ? ksamp : nrest;
+    if (m <= 0) return 0;
+    if (ndet + m > s->k_max) return -3;
+    char* in_det = (char*)calloc((size_t)n, 1);
+    keyed* rest = (keyed*)malloc(sizeof(keyed) * (size_t)n);
+    int32_t* merged = (int32_t*)malloc(sizeof(int32_t) * (size_t)(ndet + m));
+    if (!in_det || !rest || !merged) { free(in_det); free(rest); free(merged); return -4; }
+    for (int t = 0; t < ndet; ++t)
+        if (idx_row[t] < n) in_det[idx_row[t]] = 1;
+    long r = (long)b * s->Hq + h, c = 0;
+    for (long p = 0; p < n; ++p)
+        if (!in_det[p]) { rest[c].key = sample_key(seed, step, r, p); rest[c].pos = (int32_t)p; ++c; }
+    qsort(rest, (size_t)c, sizeof(keyed), by_key_then_pos);
+    for (int t = 0; t < ndet; ++t) merged[t] = idx_row[t];
+    for (long t = 0; t < m; ++t) merged[ndet + t] = rest[t].pos | SAMPLED_FLAG;
+    /* ascending by position (the flag bit does not take part in the order) */
+    for (long i = 1; i < ndet + m; ++i) {
+        int32_t v = merged[i];
+        long j = i - 1;
+        while (j >= 0 && (merged[j] & POS_MASK) > (v & POS_MASK)) { merged[j + 1] = merged[j]; --j; }
+        merged[j + 1] = v;
+    }
+    for (long t = 0; t < ndet + m; ++t) idx_row[t] = merged[t];
+    free(in_det);
+    free(rest);
+    free(merged);
+    return 0;
+}
+
+int oracle_stochastic_topk(int B, int Hq, int Hkv, int d, int P, int max_pages, int num_pages, int k_max,
+                           const uint16_t* q, const uint16_t* K, const int32_t* page_table, const int32_t* lens,
+                           const int32_t* k_det, const int32_t* k_samp, uint64_t seed, uint32_t step,
+                           int32_t* idx) {
+    oshape s = {B, Hq, Hkv, d, P, max_pages, k_max, num_pages};
+    if (check_shape(&s)) return -1;
+    for (int b = 0; b < B; ++b) {
+        if (req_len(&s, lens, b) < 0) return -1;
+        if (k_det[b] < 1 || k_samp[b] < 0) return -1;
+        if ((long)lens[b] > (long)POS_MASK) return -1;
+    }
+    int rc_all = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(min : rc_all)
+    for (long bh = 0; bh < (long)B * Hq; ++bh) {
+        int b = (int)(bh / Hq), h = (int)(bh % Hq);
+        int rc = stochastic_one(&s, q, K, page_table, b, h, lens[b], k_det[b], k_samp[b], seed, step,
+                                idx + bh * (long)k_max);
         if (rc < rc_all) rc_all = rc;
     }
     return rc_all;

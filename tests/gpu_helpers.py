@@ -136,24 +136,39 @@ def group_subproblem(w: wl.Workload, b: int, kvh: int):
     return sub
 
 
-def sampled_parity(w: wl.Workload, idx: torch.Tensor, out: torch.Tensor, groups, dense: torch.Tensor | None = None):
-    """Parity on sampled (b, kvh) groups of a large GPU workload."""
+def request_subproblem(w: wl.Workload, b: int):
+    """Request b of a GPU workload as a one-request CPU workload with a contiguous cache (data
+    movement only): its q, all its KV heads' K/V rows in logical order, an identity page table."""
+    n = int(w.lens[b])
+    P = w.P
+    npages = max(1, (n + P - 1) // P)
+    pages = w.page_table[b, :npages].long()
+    return wl.Workload(name=f"{w.name}[{b}]", B=1, Hq=w.Hq, Hkv=w.Hkv, d=w.d, P=P, max_pages=npages,
+                       num_pages=npages, k_max=w.k_max, q=w.q[b:b + 1].contiguous().cpu(),
+                       K=w.K[pages].contiguous().cpu(), V=w.V[pages].contiguous().cpu(),
+                       page_table=torch.arange(npages, dtype=torch.int32).view(1, npages),
+                       lens=torch.tensor([n], dtype=torch.int32), k=w.k[b:b + 1].cpu())
+
+
+def all_requests_parity(w: wl.Workload, idx: torch.Tensor, out: torch.Tensor, dense: torch.Tensor | None = None,
+                        requests=None):
+    """Parity of every (request, query head) row of a full-size GPU workload, one request at a time:
+    the oracle's index set and its attention over the GPU's own rows (and dense attention)."""
     idx_np = idx.cpu().numpy()
     out_np = out.cpu().numpy()
     dense_np = dense.cpu().numpy() if dense is not None else None
-    stats = []
-    for (b, kvh) in groups:
-        sub = group_subproblem(w, b, kvh)
-        G = w.G
-        rows = idx_np[b:b + 1, kvh * G:(kvh + 1) * G]
+    stats, n_diff = [], 0
+    for b in (range(w.B) if requests is None else requests):
+        sub = request_subproblem(w, b)
         shape = sub.shape()
+        rows = idx_np[b:b + 1]
         ref = oracle.topk(shape, sub.q, sub.K, sub.page_table, sub.lens, sub.k)
-        check_index_rows(rows, ref, sub.lens, sub.k,
-                         lambda bb, h: oracle.scores(shape, sub.q, sub.K, sub.page_table, sub.lens, bb, h),
-                         [(0, g) for g in range(G)])
+        n_diff += check_index_rows(rows, ref, sub.lens, sub.k,
+                                   lambda bb, h: oracle.scores(shape, sub.q, sub.K, sub.page_table, sub.lens, bb, h),
+                                   [(0, h) for h in range(w.Hq)])
         o = oracle.attend(shape, sub.q, sub.K, sub.V, sub.page_table, sub.lens, rows)
-        stats.append(check_outputs(out_np[b:b + 1, kvh * G:(kvh + 1) * G], o))
+        stats.append(check_outputs(out_np[b:b + 1], o))
         if dense_np is not None:
             od = oracle.dense(shape, sub.q, sub.K, sub.V, sub.page_table, sub.lens)
-            stats.append(check_outputs(dense_np[b:b + 1, kvh * G:(kvh + 1) * G], od))
-    return stats
+            stats.append(check_outputs(dense_np[b:b + 1], od))
+    return stats, n_diff

@@ -14,6 +14,7 @@ import pytest
 import oracle
 from tests import test_oracle as pins
 from tests import test_oracle_quest as quest_pins
+from tests import test_oracle_stochastic as stochastic_pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
 
@@ -30,8 +31,8 @@ MUTANTS = [
     ("slot_from_wrong_axis", "long slot = p % s->P;", "long slot = (p / s->P) % s->P;"),
     ("drop_first_dim", "for (int j = 0; j < s->d; ++j) acc += bf16_to_double(qh[j]) * bf16_to_double(krow[j]);\n        out[i]",
      "for (int j = 1; j < s->d; ++j) acc += bf16_to_double(qh[j]) * bf16_to_double(krow[j]);\n        out[i]"),
-    ("no_normalisation", "for (int j = 0; j < s->d; ++j) out[j] /= denom;", ""),
-    ("sign_flip_in_exponent", "double w = exp(z[t] - zmax);", "double w = exp(zmax - z[t]);"),
+    ("no_normalisation", "for (int j = 0; j < s->d; ++j) out[j] /= den;", ""),
+    ("sign_flip_in_exponent", "double e = exp(z[t] - zref)", "double e = exp(zref - z[t])"),
     ("one_row_short", "for (int i = 0; i < take; ++i) idx_row[i] = all[i].pos;",
      "for (int i = 0; i + 1 < take; ++i) idx_row[i] = all[i].pos;"),
     ("unsorted_output", "qsort(idx_row, (size_t)take, sizeof(int32_t), by_pos);", ""),
@@ -44,6 +45,15 @@ MUTANTS = [
     ("quest_budget_rounds_down", "long kp = ((long)kb + s->P - 1) / s->P;", "long kp = (long)kb / s->P;"),
     ("quest_current_page_outside_budget", "for (long t = 0; t + 1 < kp; ++t) keep[other[t].pos] = 1;",
      "for (long t = 0; t < kp && t + 1 < np; ++t) keep[other[t].pos] = 1;"),
+    # stochastic selection
+    ("sample_weight_inverted", "double w = nsamp > 0 ? (double)(n - (nsel - nsamp)) / (double)nsamp : 1.0;",
+     "double w = nsamp > 0 ? (double)nsamp / (double)(n - (nsel - nsamp)) : 1.0;"),
+    ("sample_weight_numerator_only", "        *den += e;\n", "        *den += exp(z[t] - zref);\n"),
+    ("sample_weight_rest_off_by_one", "double w = nsamp > 0 ? (double)(n - (nsel - nsamp)) / (double)nsamp : 1.0;",
+     "double w = nsamp > 0 ? (double)(n - 1 - (nsel - nsamp)) / (double)nsamp : 1.0;"),
+    ("sample_drawn_from_all_rows", "        if (!in_det[p]) { rest[c].key", "        if (1) { rest[c].key"),
+    ("sample_largest_keys", "if (x->key != y->key) return (x->key < y->key) ? -1 : 1;",
+     "if (x->key != y->key) return (x->key > y->key) ? -1 : 1;"),
     ("quest_first_dim_dropped", "for (int e = 0; e < s->d && rc == 0; ++e) {\n            double qe",
      "for (int e = 1; e < s->d && rc == 0; ++e) {\n            double qe"),
 ]
@@ -64,6 +74,13 @@ PINS = [
     quest_pins.test_ties_go_to_lower_page_and_budget_rounds_up,
     quest_pins.test_partial_last_page_and_whole_cache_budget,
     quest_pins.test_selection_is_the_most_relevant_pages,
+    stochastic_pins.test_splitmix64_published_outputs,
+    stochastic_pins.test_zero_samples_is_exact_topk,
+    stochastic_pins.test_sampling_all_the_rest_is_dense_attention,
+    stochastic_pins.test_weighted_sums_are_unbiased_over_every_sample,
+    stochastic_pins.test_sample_is_distinct_outside_the_deterministic_rows_and_reproducible,
+    stochastic_pins.test_each_rest_row_is_drawn_with_probability_m_over_rest,
+    stochastic_pins.test_sample_is_the_rows_with_the_smallest_keys,
 ]
 
 

@@ -1,8 +1,8 @@
 """GPU parity: the CUDA path through the C ABI against the fp64 CPU oracle on the same seeded inputs.
 
-Small cases are compared element by element on every (b, h); the full-size workloads (the five
-named configurations) run in the launch configuration the benchmark times and are compared on
-sampled (request, KV head) groups.  Rules and tolerances: tests/gpu_helpers.py.
+Small cases and the full-size workloads (the five named configurations, in the launch
+configuration the benchmark times) are compared element by element on every (b, h) row; the
+full-size ones one request at a time.  Rules and tolerances: tests/gpu_helpers.py.
 """
 from __future__ import annotations
 
@@ -245,26 +245,28 @@ def _big(name, **kw):
     return w, gh.Runner(w)
 
 
-def test_long128k_sampled():
+def test_long128k_all_groups():
+    """Long-context workload (B = 4, 64/8 heads, N = 131072, k = 2621), in the launch configuration
+    the benchmark times: every (request, head) row against the oracle, sparse and dense decode."""
     w, r = _big("long128k")
     idx = r.topk()
     out = r.sparse(idx)
     dense = r.dense()
     assert r.device_status() == 0
-    gh.sampled_parity(w, idx, out, [(0, 0), (1, 3), (2, 5), (3, 7)], dense=dense)
-    # attention sinks: K rows 0-3 are scaled by 3, so a head whose q is aligned with them keeps them;
-    # at least the index rows must all be full
+    gh.all_requests_parity(w, idx, out, dense=dense)
+    # attention sinks: K rows 0-3 are scaled by 3; every index row is full
     assert (idx[:, :, :2621] >= 0).all()
 
 
 @pytest.mark.parametrize("ratio", [10, 50, 100, 1])
-def test_sweep128k_sampled(ratio):
+def test_sweep128k_all_groups(ratio):
+    """Sparsity sweep (B = 16, 32/8 heads, N = 131072, k = N/10, N/50, N/100, N): every row."""
     w, r = _big("sweep128k", ratio=ratio)
     idx = r.topk()
     out = r.sparse(idx)
     dense = r.dense() if ratio == 1 else None
     assert r.device_status() == 0
-    gh.sampled_parity(w, idx, out, [(0, 0), (15, 7)], dense=dense)
+    gh.all_requests_parity(w, idx, out, dense=dense)
     if ratio == 1:
         # k = N: both read every row; the sparse decode sums per head and the dense one per GQA
         # group, in different segment orders, so only fp32 rounding (and the bf16 hi + lo split of
@@ -273,6 +275,8 @@ def test_sweep128k_sampled(ratio):
 
 
 def test_ragged_steps_with_append():
+    """Ragged agentic batch (32 requests, N_b in [8192, 163840], k_b = N_b / 50) over 64 decode steps
+    with one K/V row appended per request per step: every row checked at steps 0, 32 and 63."""
     w, r = _big("ragged")
     steps = w.meta["steps"]
     ratio = w.meta["ratio"]
@@ -287,7 +291,7 @@ def test_ragged_steps_with_append():
             assert r.device_status() == 0
             lens = w.lens.cpu()
             assert int(w.k[0]) == wl.k_for_ratio(int(lens[0]), ratio)
-            gh.sampled_parity(w, idx, out, [(0, 0), (int(torch.argmax(lens)), 3), (int(torch.argmin(lens)), 6)])
+            gh.all_requests_parity(w, idx, out)
     assert r.device_status() == 0
 
 
