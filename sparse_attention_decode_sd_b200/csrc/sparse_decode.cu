@@ -268,7 +268,11 @@ __device__ __forceinline__ int warp_inclusive_scan(int v) {
 __global__ void __launch_bounds__(1024, 2) rows_kernel(DecodeArgs a) {
     __shared__ int s_neg[32];   // per warp: first negative entry it saw
     __shared__ int s_len[32];   // per row of this CTA
-    pdl_enter();
+    // The decode kernel is released only after this wait: when its grid starts, all earlier work in
+    // the stream (the indexer writing idx, anything writing q, K, V or the page table) is complete, so
+    // it may read idx before its own wait, which it needs only for the row lengths and counters.
+    pdl_wait();
+    pdl_launch_dependents();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int tpr = a.tpr, wpr = tpr >> 5;
     const int rl = tid / tpr, t = tid - rl * tpr;
@@ -358,6 +362,7 @@ struct RowWalker {
     int pt_off;          // b * max_pages: row r's request in the page table
     int kvh;             // KV head of row r
     const int32_t* ix;   // idx of row r, indexed by global entry
+    bool full;           // every row holds k_max entries (row lengths need no lookup)
     bool seg_new;        // the next tile opens a segment
     int seq;             // tiles handed out so far
 };
@@ -373,7 +378,7 @@ __device__ __forceinline__ void enter_row(const DecodeArgs& a, RowWalker& w, int
     w.kvh = (r - b * a.Hq) / a.G;
     w.pt_off = b * a.max_pages;
     w.ix = a.idx + (long)r * a.k_max - rstart;
-    w.next_len = r + 1 < R ? __ldg(a.rlen + r + 1) : 0;
+    w.next_len = r + 1 < R ? (w.full ? a.k_max : __ldg(a.rlen + r + 1)) : 0;
     w.seg_new = true;
 }
 
@@ -408,7 +413,7 @@ __device__ __forceinline__ RowTile next_row_tile(const DecodeArgs& a, RowWalker&
     }
     int flags = w.seg_new ? kFlagFirst : 0;
     w.seg_new = false;
-    if (lane < rows) d.v = __ldg(w.ix + w.e + lane);
+    if (lane < rows) d.v = __ldcg(w.ix + w.e + lane);   // L2: idx may be read before this grid's wait
     w.e += rows;
     if (w.e == w.rend || w.e == w.e_end) {
         flags |= kFlagLast;
@@ -429,8 +434,8 @@ __device__ __forceinline__ RowTile next_row_tile(const DecodeArgs& a, RowWalker&
 // inside the page-table row (below max_pages * 16) are looked up.
 __device__ __forceinline__ void lookup_pages(const DecodeArgs& a, RowTile& d) {
     const int lane = threadIdx.x & 31;
-    if (d.v >= 0 && d.v < a.n_cap) d.page = __ldg(a.page_table + d.pt_off + (d.v >> 4));
-    if ((d.hdr >> 5) & kFlagFirst) d.q2 = __ldg(reinterpret_cast<const uint2*>(a.q + (long)d.r * kHeadDim) + lane);
+    if (d.v >= 0 && d.v < a.n_cap) d.page = __ldcg(a.page_table + d.pt_off + (d.v >> 4));
+    if ((d.hdr >> 5) & kFlagFirst) d.q2 = __ldcg(reinterpret_cast<const uint2*>(a.q + (long)d.r * kHeadDim) + lane);
 }
 
 // 4-row gather of 128-byte half rows (2-D tensor [cache rows][128 dims], box {64, 1}) into shared
@@ -618,7 +623,8 @@ __device__ __forceinline__ void merge_row(const DecodeArgs& a, int r, int nseg) 
         make_float4(o4.x * inv, o4.y * inv, o4.z * inv, o4.w * inv);
 }
 
-// End of this warp's segment of row r.
+// End of this warp's segment of row r: a row held by one warp is written out; otherwise the
+// partial is stored, its arrival counted, and the last of the row's warps to arrive merges them.
 __device__ __forceinline__ void finish_row_segment(const DecodeArgs& a, int r, int j, int nseg, const HeadState& st) {
     const int lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
     float l = st.l;
@@ -669,73 +675,11 @@ __global__ void __launch_bounds__(32) sparse_decode_kernel(DecodeArgs a, const _
         mbar_fence_init();
     }
     __syncwarp();
-    pdl_enter();
+    pdl_launch_dependents();
 
     const int R = a.B * a.Hq;
-    // E = all entries: the length sums of the rows_kernel CTAs, each lane summing kPrologue
-    // consecutive ones per round
-    int E = 0;
-    for (int base = 0; base < a.nb; base += 32 * kPrologue) {
-        const int k0 = base + kPrologue * lane;
-#pragma unroll
-        for (int i = 0; i < kPrologue; ++i) E += k0 + i < a.nb ? __ldg(a.bsum + k0 + i) : 0;
-    }
-    E = __reduce_add_sync(0xffffffffu, E);
-    if (E == 0) return;
     RowWalker w;
-    w.epw = max(a.min_epw, (int)(((long)E + a.total_warps - 1) / a.total_warps));
-    const long e0 = (long)blockIdx.x * w.epw;
-    if (e0 >= E) return;
-    w.e = (int)e0;
-    w.e_end = (int)min((long)E, e0 + w.epw);
-    // the rows_kernel CTA whose rows hold entry w.e: one scan of the lanes' sums per round (the
-    // sums are in L1 now), then the lane that holds it walks its kPrologue sums
-    int blk = -1, blk0 = 0, blen = 0;
-    {
-        int acc = 0;
-        for (int base = 0; base < a.nb && blk < 0; base += 32 * kPrologue) {
-            const int k0 = base + kPrologue * lane;
-            int v[kPrologue], sum = 0;
-#pragma unroll
-            for (int i = 0; i < kPrologue; ++i) {
-                v[i] = k0 + i < a.nb ? __ldg(a.bsum + k0 + i) : 0;
-                sum += v[i];
-            }
-            const int incl = warp_inclusive_scan(sum);
-            const uint32_t hit = __ballot_sync(0xffffffffu, acc + incl > w.e);
-            if (hit != 0u) {
-                const int l = __ffs(hit) - 1;
-                int c = acc + incl - sum, kb = -1, kb0 = 0, kl = 0;   // lane l: its sums in order
-#pragma unroll
-                for (int i = 0; i < kPrologue; ++i) {
-                    if (kb < 0 && c + v[i] > w.e) {
-                        kb = k0 + i;
-                        kb0 = c;
-                        kl = v[i];
-                    }
-                    c += v[i];
-                }
-                blk = __shfl_sync(0xffffffffu, kb, l);
-                blk0 = __shfl_sync(0xffffffffu, kb0, l);
-                blen = __shfl_sync(0xffffffffu, kl, l);
-            }
-            acc += __shfl_sync(0xffffffffu, incl, 31);
-        }
-    }
-    if (blk < 0) return;   // not reached: w.e < E
-    if (a.rpc == 1) {      // one row per CTA of the row pass
-        enter_row(a, w, blk, blk0, blen);
-    } else {
-        const int r0 = blk * a.rpc;
-        const int v = (lane < a.rpc && r0 + lane < R) ? __ldg(a.rlen + r0 + lane) : 0;
-        const int incl = warp_inclusive_scan(v);
-        const uint32_t hit = __ballot_sync(0xffffffffu, blk0 + incl > w.e);
-        if (hit == 0u) return;   // not reached: the CTA's rows hold entry w.e
-        const int l = __ffs(hit) - 1;
-        enter_row(a, w, r0 + l, blk0 + __shfl_sync(0xffffffffu, incl - v, l), __shfl_sync(0xffffffffu, v, l));
-    }
     w.seq = 0;
-
     // this lane's ldmatrix offsets inside a 2 KB half block: K (A operand, rows 8 (lane>>3 & 1) +
     // (lane & 7), chunk 2 (j & 3) + (lane >> 4)) and V (A operand transposed, rows 8 (lane >> 4) +
     // (lane & 7), chunk 2 (mt & 3) + (lane >> 3 & 1)), each chunk swizzled by the row's low 3 bits
@@ -749,27 +693,143 @@ __global__ void __launch_bounds__(32) sparse_decode_kernel(DecodeArgs a, const _
         }
     }
     const uint32_t kv0 = smem_addr(ws.kv);
-
+    RowTile dA, dB, dC;   // the pipeline's tile records (see the main loop)
+    auto start_pipeline = [&]() {
+        dA = next_row_tile(a, w);
+        dB = next_row_tile(a, w);
+        dC = next_row_tile(a, w);
+        lookup_pages(a, dA);
+        issue_row_tile(a, ws, kv0, dA, &kmap, &vmap);   // the walk's first tile
+        dA = dB;
+        dB = dC;
+        dC = next_row_tile(a, w);
+        lookup_pages(a, dA);
+    };
+    // Speculative start on the split that holds when every row has k_max entries (the indexer's
+    // rows, the common case): the first tile is gathered while rows_kernel still runs.  After the
+    // wait, the true entry count decides: equal to R * k_max, the split is the same and the walk
+    // goes on; otherwise the speculative tile is drained and the walk restarts on the row lengths.
+    const long e_full = (long)R * a.k_max;   // < 2^31 (checked on the host)
+    w.full = true;
+    w.epw = max(a.min_epw, (int)((e_full + a.total_warps - 1) / a.total_warps));
+    const bool spec = (long)blockIdx.x * w.epw < e_full;
+    if (spec) {
+        w.e = (int)blockIdx.x * w.epw;
+        w.e_end = (int)min(e_full, (long)w.e + w.epw);
+        const int r = w.e / a.k_max;
+        enter_row(a, w, r, r * a.k_max, a.k_max);
+        start_pipeline();
+    }
+    pdl_wait();   // rows_kernel: row lengths, checks, zeroed arrival counters
+    // E = all entries: the length sums of the rows_kernel CTAs, each lane summing kPrologue
+    // consecutive ones per round
+    int E = 0;
+    for (int base = 0; base < a.nb; base += 32 * kPrologue) {
+        const int k0 = base + kPrologue * lane;
+#pragma unroll
+        for (int i = 0; i < kPrologue; ++i) E += k0 + i < a.nb ? __ldg(a.bsum + k0 + i) : 0;
+    }
+    E = __reduce_add_sync(0xffffffffu, E);
+    int t = 0;   // the tile the main loop consumes first
+    // A speculative tile that is not used is left to complete while the walk restarts at tile 1;
+    // stage 0 is waited for before its next use or before the warp exits.
+    bool spec_pending = false;
+    auto drain_spec = [&]() -> bool {
+        if (!spec_pending) return true;
+        spec_pending = false;
+        const bool done = __all_sync(0xffffffffu, mbar_wait(&ws.full[0], 0u));
+        if (!done && lane == 0) report(a.status, SD_ERR_TIMEOUT);
+        return done;
+    };
+    if (!(spec && E == e_full)) {
+        if (spec) {
+            spec_pending = true;
+            t = 1;
+        }
+        if (E == 0) {
+            drain_spec();
+            return;
+        }
+        w.full = false;
+        w.epw = max(a.min_epw, (int)(((long)E + a.total_warps - 1) / a.total_warps));
+        const long e0 = (long)blockIdx.x * w.epw;
+        if (e0 >= E) {
+            drain_spec();
+            return;
+        }
+        w.e = (int)e0;
+        w.e_end = (int)min((long)E, e0 + w.epw);
+        // the rows_kernel CTA whose rows hold entry w.e: one scan of the lanes' sums per round (the
+        // sums are in L1 now), then the lane that holds it walks its kPrologue sums
+        int blk = -1, blk0 = 0, blen = 0;
+        {
+            int acc = 0;
+            for (int base = 0; base < a.nb && blk < 0; base += 32 * kPrologue) {
+                const int k0 = base + kPrologue * lane;
+                int v[kPrologue], sum = 0;
+#pragma unroll
+                for (int i = 0; i < kPrologue; ++i) {
+                    v[i] = k0 + i < a.nb ? __ldg(a.bsum + k0 + i) : 0;
+                    sum += v[i];
+                }
+                const int incl = warp_inclusive_scan(sum);
+                const uint32_t hit = __ballot_sync(0xffffffffu, acc + incl > w.e);
+                if (hit != 0u) {
+                    const int l = __ffs(hit) - 1;
+                    int c = acc + incl - sum, kb = -1, kb0 = 0, kl = 0;   // lane l: its sums in order
+#pragma unroll
+                    for (int i = 0; i < kPrologue; ++i) {
+                        if (kb < 0 && c + v[i] > w.e) {
+                            kb = k0 + i;
+                            kb0 = c;
+                            kl = v[i];
+                        }
+                        c += v[i];
+                    }
+                    blk = __shfl_sync(0xffffffffu, kb, l);
+                    blk0 = __shfl_sync(0xffffffffu, kb0, l);
+                    blen = __shfl_sync(0xffffffffu, kl, l);
+                }
+                acc += __shfl_sync(0xffffffffu, incl, 31);
+            }
+        }
+        if (blk < 0) {   // not reached: w.e < E
+            drain_spec();
+            return;
+        }
+        if (a.rpc == 1) {      // one row per CTA of the row pass
+            enter_row(a, w, blk, blk0, blen);
+        } else {
+            const int r0 = blk * a.rpc;
+            const int v = (lane < a.rpc && r0 + lane < R) ? __ldg(a.rlen + r0 + lane) : 0;
+            const int incl = warp_inclusive_scan(v);
+            const uint32_t hit = __ballot_sync(0xffffffffu, blk0 + incl > w.e);
+            if (hit == 0u) {   // not reached: the CTA's rows hold entry w.e
+                drain_spec();
+                return;
+            }
+            const int l = __ffs(hit) - 1;
+            enter_row(a, w, r0 + l, blk0 + __shfl_sync(0xffffffffu, incl - v, l), __shfl_sync(0xffffffffu, v, l));
+        }
+        w.seq = t;
+        start_pipeline();
+    }
     // Software pipeline over tiles, so that no load but the gather itself is waited for: while tile
     // t is consumed, tile t + 1 is gathered (its pages were looked up a step earlier), the pages of
     // tile t + 2 are looked up (its positions were loaded two steps earlier) and the positions of
-    // tile t + 4 are loaded.
-    static_assert(kSparseStages == 2, "the pipeline below gathers one tile ahead");
-    // (Each page lookup follows the rotation of the records, so that no record is copied while a
-    // load into it is in flight: such a register copy would wait for the load.)
-    RowTile dA = next_row_tile(a, w), dB = next_row_tile(a, w), dC = next_row_tile(a, w);
-    lookup_pages(a, dA);
-    issue_row_tile(a, ws, kv0, dA, &kmap, &vmap);   // tile 0
-    dA = dB;
-    dB = dC;
-    dC = next_row_tile(a, w);
-    lookup_pages(a, dA);
+    // tile t + 4 are loaded.  (Each page lookup follows the rotation of the records, so that no
+    // record is copied while a load into it is in flight: such a register copy would wait for the
+    // load.)
+    static_assert(kSparseStages == 2, "the pipeline gathers one tile ahead");
     HeadState st;
     reset_head(st);
     bool ok = true;
-    int t = 0;
     for (;; ++t) {
         const int stage = t & (kSparseStages - 1);
+        if (spec_pending && ((dA.hdr >> 8) & (kSparseStages - 1)) == 0 && !drain_spec()) {
+            ok = false;
+            break;
+        }
         issue_row_tile(a, ws, kv0, dA, &kmap, &vmap);   // into the stage tile t - 1 used
         dA = dB;
         dB = dC;
@@ -790,6 +850,7 @@ __global__ void __launch_bounds__(32) sparse_decode_kernel(DecodeArgs a, const _
         }
         __syncwarp();   // every lane has read the stage before it is refilled
     }
+    drain_spec();
     if (!ok) {
         // A copy never completed: record it, wait (bounded) for this warp's copies still in
         // flight, and return; the rows this warp held are left unwritten.
