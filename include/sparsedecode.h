@@ -128,7 +128,10 @@ SD_API sd_status sd_topk_select(const sd_shape* shape, const int32_t* lens, cons
  *   64 query heads at 131072 positions and k_max 2621 fits), else SD_ERR_WORKSPACE and nothing is
  *   launched.
  *   The first call on a device looks up the array's device address (cudaGetSymbolAddress) with that
- *   device current; make that first call before any stream capture.
+ *   device current and keeps it; make that first call before any stream capture.  The address
+ *   belongs to the device's current context: after cudaDeviceReset the library's device code is
+ *   loaded again and the kept address is no longer valid, so do not call this entry point after a
+ *   cudaDeviceReset in the same process.
  *   Every call on a device uses the same array, which keeps the last call's scores: calls whose
  *   kernels overlap on the GPU (other streams, other host threads) race and must be serialised by
  *   the caller. */
@@ -142,12 +145,51 @@ SD_API sd_status sd_topk_index_static(const sd_shape* shape, const void* q, cons
  *   S = the entries of idx[b][h] before its first negative one.  An empty S gives out = 0.
  *   Each query head gathers its own rows; the heads of a GQA group are processed side by side, so a
  *   row that several of them selected is read from HBM about once and from L2 after that.
+ *   The call launches two kernels; the second starts gathering before the first (the row checks)
+ *   ends, so idx, q, K, V and the page table must be complete when the call is enqueued (stream
+ *   order), as for every call of the library.
+ *   num_pages * 16 * Hkv must be below 2^31 (cache rows are TMA coordinates), else
+ *   SD_ERR_UNSUPPORTED.
  *   Device checks: entries must be < N_b and map to a page-table entry in range (SD_ERR_INDEX_OOB),
  *   strictly ascending, with nothing but padding after the first negative entry (SD_ERR_ORDER).
  *   B * Hq * k_max must be below 2^31 (else SD_ERR_UNSUPPORTED, also from sd_workspace_size). */
 SD_API sd_status sd_sparse_decode(const sd_shape* shape, const void* q, const void* K, const void* V,
                            const int32_t* page_table, const int32_t* lens, const int32_t* idx, float* out,
                            void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/* Stochastic index selection, the vAttention-style selection the pages evaluate ("Technische
+ * Zusammenfassung: Kontextsparsitaet bei der Inferenzzeit", sec. 2 "Stochastische Indexierung" and
+ * sec. 3A "Stochastisch vs. Deterministisch"; the pages name the method, not its estimator, and the
+ * reading implemented here is stated in full in the library's documentation):
+ *   per (b, h): S_d = the exact top-k_det[b] rows (as sd_topk_index with k = k_det), plus
+ *   m = min(k_samp[b], |R|) rows drawn uniformly without replacement from the rest
+ *   R = [0, N_b) \ S_d.  Position p of R gets the key u(p) = top 32 bits of
+ *   SM(SM(SM(seed + step) + b * Hq + h) + p), SM(x) being one SplitMix64 output from state x (a
+ *   counter-based generator, so the draw is reproducible), and the m positions with the smallest
+ *   (u, p) are drawn.
+ *   idx[b][h] holds S_d and the drawn rows together in ascending position, each drawn row with
+ *   SD_SAMPLED_FLAG (bit 30) set on its position, then -1; sd_sparse_decode_sampled weighs each drawn
+ *   row by |R| / m.  k_det[b] >= 1 and k_samp[b] >= 0 (device array [B]); shape->k_max must hold
+ *   k_det + k_samp rows of every request (else the row is left as S_d and dev_status records
+ *   SD_ERR_INVALID_ARG).  Workspace: sd_workspace_size(shape, SD_OP_TOPK).  SD_ERR_UNSUPPORTED when
+ *   the row bitmaps and candidates of max_pages_per_req * 16 positions do not fit one SM's shared
+ *   memory (above about 600K positions per request). */
+#define SD_SAMPLED_FLAG 0x40000000
+SD_API sd_status sd_stochastic_index(const sd_shape* shape, const void* q, const void* K, const int32_t* page_table,
+                                     const int32_t* lens, const int32_t* k_det, const int32_t* k_samp,
+                                     uint64_t seed, uint32_t step, int32_t* idx, void* workspace,
+                                     size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/* sd_sparse_decode over the rows of a stochastic selection: an entry with SD_SAMPLED_FLAG is a drawn
+ * row and its exp(z) counts w = (N_b - plain entries) / drawn entries times, in both the numerator and
+ * the denominator of the softmax -- the inverse of its inclusion probability, so that the drawn rows
+ * estimate the sums over all rows outside S_d without bias.  Without flagged entries the result is
+ * that of sd_sparse_decode.  Positions are the entries' low 30 bits; the checks of sd_sparse_decode
+ * apply to them.  Workspace: sd_workspace_size(shape, SD_OP_SPARSE). */
+SD_API sd_status sd_sparse_decode_sampled(const sd_shape* shape, const void* q, const void* K, const void* V,
+                                          const int32_t* page_table, const int32_t* lens, const int32_t* idx,
+                                          float* out, void* workspace, size_t workspace_bytes,
+                                          int32_t* dev_status, void* stream);
 
 /* Dense decode attention over all N_b rows ("Dense" mode of Fig. 1(a)); the comparator of the
  * sparse kernel at the same shape.  shape->k_max is ignored. */

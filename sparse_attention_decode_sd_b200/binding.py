@@ -29,9 +29,12 @@ SD_OP_SPARSE = 2
 SD_OP_DENSE = 3
 SD_OP_QUEST = 4
 
+SD_SAMPLED_FLAG = 1 << 30   # idx entry of a row drawn by sd_stochastic_index (position in the low 30 bits)
+
 EXPORTED = ("sd_workspace_size", "sd_topk_index", "sd_topk_scores", "sd_topk_select", "sd_topk_index_static",
-            "sd_sparse_decode", "sd_dense_decode", "sd_append_kv", "sd_quest_summarize", "sd_quest_index",
-            "sd_selftest_wait_timeout", "sd_status_string", "sd_last_cuda_error", "sd_version")
+            "sd_sparse_decode", "sd_stochastic_index", "sd_sparse_decode_sampled", "sd_dense_decode", "sd_append_kv",
+            "sd_quest_summarize", "sd_quest_index", "sd_selftest_wait_timeout", "sd_status_string",
+            "sd_last_cuda_error", "sd_version")
 
 
 class SdShape(ctypes.Structure):
@@ -72,6 +75,8 @@ def load():
     lib.sd_topk_index_static.argtypes = [SH, P, P, P, P, P, P, P, P]
     lib.sd_topk_index_static.restype = I32
     lib.sd_sparse_decode.argtypes = [SH, P, P, P, P, P, P, P, P, SZ, P, P]
+    lib.sd_sparse_decode_sampled.argtypes = [SH, P, P, P, P, P, P, P, P, SZ, P, P]
+    lib.sd_stochastic_index.argtypes = [SH, P, P, P, P, P, P, ctypes.c_uint64, ctypes.c_uint32, P, P, SZ, P, P]
     lib.sd_dense_decode.argtypes = [SH, P, P, P, P, P, P, P, SZ, P, P]
     lib.sd_append_kv.argtypes = [SH, P, P, P, P, P, P, P, I32, P, P]
     lib.sd_quest_summarize.argtypes = [SH, P, P, P, P, I32, P, P]
@@ -79,7 +84,8 @@ def load():
     lib.sd_selftest_wait_timeout.argtypes = [ctypes.c_uint32, P, P]
     lib.sd_selftest_wait_timeout.restype = I32
     for f in (lib.sd_workspace_size, lib.sd_topk_index, lib.sd_topk_scores, lib.sd_topk_select, lib.sd_sparse_decode,
-              lib.sd_dense_decode, lib.sd_append_kv, lib.sd_quest_summarize, lib.sd_quest_index):
+              lib.sd_sparse_decode_sampled, lib.sd_stochastic_index, lib.sd_dense_decode, lib.sd_append_kv,
+              lib.sd_quest_summarize, lib.sd_quest_index):
         f.restype = I32
     lib.sd_status_string.argtypes = [I32]
     lib.sd_status_string.restype = ctypes.c_char_p
@@ -167,7 +173,7 @@ def sd_topk_select(shape, lens, k, idx, workspace, dev_status, stream=None, chec
 
 
 def sd_topk_index_static(shape, q, K, page_table, lens, k, idx, dev_status, stream=None, check=True) -> int:
-    """sd_topk_index with the library's own static 32 MiB score scratch (no workspace argument)."""
+    """sd_topk_index with the library's own static 48 MiB scratch (no workspace argument)."""
     st = load().sd_topk_index_static(ctypes.byref(shape), _ptr(q), _ptr(K), _ptr(page_table), _ptr(lens), _ptr(k),
                                      _ptr(idx), _ptr(dev_status), _stream(stream))
     return _check(st, "sd_topk_index_static", check)
@@ -179,6 +185,23 @@ def sd_sparse_decode(shape, q, K, V, page_table, lens, idx, out, workspace, dev_
                                  _ptr(idx), _ptr(out), _ptr(workspace), _ws_bytes(workspace), _ptr(dev_status),
                                  _stream(stream))
     return _check(st, "sd_sparse_decode", check)
+
+
+def sd_stochastic_index(shape, q, K, page_table, lens, k_det, k_samp, seed, step, idx, workspace, dev_status,
+                        stream=None, check=True) -> int:
+    st = load().sd_stochastic_index(ctypes.byref(shape), _ptr(q), _ptr(K), _ptr(page_table), _ptr(lens), _ptr(k_det),
+                                    _ptr(k_samp), ctypes.c_uint64(int(seed) & 0xFFFFFFFFFFFFFFFF),
+                                    ctypes.c_uint32(int(step) & 0xFFFFFFFF), _ptr(idx), _ptr(workspace),
+                                    _ws_bytes(workspace), _ptr(dev_status), _stream(stream))
+    return _check(st, "sd_stochastic_index", check)
+
+
+def sd_sparse_decode_sampled(shape, q, K, V, page_table, lens, idx, out, workspace, dev_status, stream=None,
+                             check=True) -> int:
+    st = load().sd_sparse_decode_sampled(ctypes.byref(shape), _ptr(q), _ptr(K), _ptr(V), _ptr(page_table),
+                                         _ptr(lens), _ptr(idx), _ptr(out), _ptr(workspace), _ws_bytes(workspace),
+                                         _ptr(dev_status), _stream(stream))
+    return _check(st, "sd_sparse_decode_sampled", check)
 
 
 def sd_dense_decode(shape, q, K, V, page_table, lens, out, workspace, dev_status, stream=None, check=True) -> int:

@@ -121,10 +121,11 @@ DenseLayout dense_layout(const Dims& d) {
 
 // sparse decode: rows_kernel shape (threads per row: enough warps for kRowBatch entries each, up to
 // 1024; CTAs of at least 256 threads when rows are short) and its workspace, in order:
-// acc [B][Hq][kRowSegs][128] fp32, ml [B][Hq][kRowSegs] float2, rlen [B*Hq], arrive [B*Hq], bsum [nb]
+// acc [B][Hq][kRowSegs][128] fp32, ml [B][Hq][kRowSegs] float2, rlen [B*Hq], arrive [B*Hq], bsum [nb],
+// rlw [B*Hq] fp32
 struct SparseLayout {
     int tpr, rpc, nb;
-    size_t acc, ml, rlen, arrive, bsum, total;
+    size_t acc, ml, rlen, arrive, bsum, rlw, total;
 };
 SparseLayout sparse_layout(const Dims& d) {
     SparseLayout L;
@@ -141,7 +142,8 @@ SparseLayout sparse_layout(const Dims& d) {
     L.rlen = L.ml + align256(slots * sizeof(float2));
     L.arrive = L.rlen + align256((size_t)rows * sizeof(int));
     L.bsum = L.arrive + align256((size_t)rows * sizeof(int));
-    L.total = L.bsum + align256((size_t)L.nb * sizeof(int));
+    L.rlw = L.bsum + align256((size_t)L.nb * sizeof(int));
+    L.total = L.rlw + align256((size_t)rows * sizeof(float));
     return L;
 }
 // entries of all rows are counted in int32
@@ -149,6 +151,8 @@ bool sparse_fits(const Dims& d) { return (long)d.B * d.Hq * d.k_max < (1L << 31)
 size_t decode_workspace(const Dims& d, bool dense) { return dense ? dense_layout(d).total : sparse_layout(d).total; }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+long d_k_max_of(const sd_shape* s) { return s ? (long)s->k_max : 0; }
 
 thread_local cudaError_t g_last_cuda_error = cudaSuccess;
 
@@ -160,7 +164,7 @@ sd_status launch_status(cudaError_t e) {
 
 sd_status decode_common(const sd_shape* shape, const void* q, const void* K, const void* V, const int32_t* page_table,
                         const int32_t* lens, const int32_t* idx, float* out, void* workspace, size_t workspace_bytes,
-                        int32_t* dev_status, void* stream, bool dense) {
+                        int32_t* dev_status, void* stream, bool dense, bool weighted = false) {
     Dims d;
     sd_status st = check_shape(shape, &d);
     if (st != SD_OK) return st;
@@ -214,6 +218,8 @@ sd_status decode_common(const sd_shape* shape, const void* q, const void* K, con
     a.rlen = reinterpret_cast<int*>(ws + L.rlen);
     a.arrive = reinterpret_cast<int*>(ws + L.arrive);
     a.bsum = reinterpret_cast<int*>(ws + L.bsum);
+    a.rlw = reinterpret_cast<float*>(ws + L.rlw);
+    a.weighted = weighted ? 1 : 0;
     a.tpr = L.tpr;
     a.rpc = L.rpc;
     a.nb = L.nb;
@@ -351,6 +357,54 @@ sd_status sd_sparse_decode(const sd_shape* shape, const void* q, const void* K, 
                            void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream) {
     return decode_common(shape, q, K, V, page_table, lens, idx, out, workspace, workspace_bytes, dev_status, stream,
                          false);
+}
+
+sd_status sd_sparse_decode_sampled(const sd_shape* shape, const void* q, const void* K, const void* V,
+                                   const int32_t* page_table, const int32_t* lens, const int32_t* idx, float* out,
+                                   void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream) {
+    return decode_common(shape, q, K, V, page_table, lens, idx, out, workspace, workspace_bytes, dev_status, stream,
+                         false, true);
+}
+
+sd_status sd_stochastic_index(const sd_shape* shape, const void* q, const void* K, const int32_t* page_table,
+                              const int32_t* lens, const int32_t* k_det, const int32_t* k_samp, uint64_t seed,
+                              uint32_t step, int32_t* idx, void* workspace, size_t workspace_bytes,
+                              int32_t* dev_status, void* stream) {
+    if (!k_samp || !aligned(k_samp, 4)) return SD_ERR_INVALID_ARG;
+    TopkArgs a;
+    DeviceInfo di;
+    sd_status st = topk_args(shape, q, K, page_table, lens, k_det, idx, workspace, workspace_bytes, dev_status, true,
+                             true, &a, &di);
+    if (st != SD_OK) return st;
+    SampleArgs sa = {};
+    sa.lens = lens;
+    sa.k_det = k_det;
+    sa.k_samp = k_samp;
+    sa.idx = idx;
+    sa.status = dev_status;
+    sa.seed = seed;
+    sa.step = step;
+    sa.B = a.B;
+    sa.Hq = a.Hq;
+    sa.k_max = a.k_max;
+    sa.n_cap = a.n_cap;
+    sa.words = (int)((a.n_cap + 31) / 32);
+    // candidates: what shared memory holds next to two position bitmaps, the radix histogram and
+    // the scan state; at least twice k_max (the threshold aims at about m + 6 sqrt(m) + 32 of them)
+    sa.cap = 0;
+    const size_t fixed = sample_smem(sa);
+    if (fixed >= kSmemBudget) return SD_ERR_UNSUPPORTED;
+    const long cap = (long)((kSmemBudget - fixed) / (sizeof(uint32_t) + 2 * sizeof(int)));
+    if (cap < 2L * d_k_max_of(shape) + 1024) return SD_ERR_UNSUPPORTED;
+    sa.cap = (int)(cap > (1 << 20) ? (1 << 20) : cap);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    st = launch_status(launch_threshold(a, s));
+    if (st != SD_OK) return st;
+    st = launch_status(launch_score_pass(a, di.sms, s));
+    if (st != SD_OK) return st;
+    st = launch_status(launch_select(a, s));
+    if (st != SD_OK) return st;
+    return launch_status(launch_sample(sa, s));
 }
 
 sd_status sd_dense_decode(const sd_shape* shape, const void* q, const void* K, const void* V,

@@ -49,6 +49,8 @@ constexpr int kMaxDecodeWarps = 1280;   // dense decode: persistent warps (one p
 constexpr int kMaxSparseWarps = 4096;   // sparse decode: persistent warps (one per CTA) at most
 constexpr int kRowSegs = 64;            // sparse decode: segment slots per (b, h) row
 constexpr int kRowBatch = 4;            // sparse decode: consecutive idx entries per rows_kernel thread and pass
+constexpr uint32_t kSampledFlag = 0x40000000u;   // idx entry: a row drawn by the stochastic selection
+constexpr int kPosMask = 0x3fffffff;             // the position bits of an idx entry
 
 struct DecodeArgs {
     const __nv_bfloat16* q;
@@ -62,6 +64,7 @@ struct DecodeArgs {
     int* rlen;            // [B*Hq] entries before the first negative one
     int* arrive;          // [B*Hq] segments of the row finished so far (zeroed by rows_kernel)
     int* bsum;            // [nb] entries of the rows of each rows_kernel CTA
+    float* rlw;           // [B*Hq] weighted mode: log2 of the weight of the row's drawn entries
     // workspace, dense decode
     int* counts;          // [nrt] rows per range
     // workspace, both
@@ -77,6 +80,8 @@ struct DecodeArgs {
     int jmax;             // segment slots per (b, h)
     int total_warps;      // persistent decode warps in the grid
     float scale_log2;     // log2(e) / sqrt(d)
+    int weighted;         // sparse: idx entries with kSampledFlag are drawn rows of a stochastic
+                          // selection, weighted by (N_b - plain entries) / drawn entries
 };
 
 size_t decode_smem();
@@ -107,6 +112,24 @@ cudaError_t launch_quest_summarize(const QuestArgs& a, cudaStream_t stream);
 cudaError_t launch_quest_score(const QuestArgs& a, cudaStream_t stream);
 cudaError_t launch_quest_select(const QuestArgs& a, cudaStream_t stream);
 size_t quest_select_smem(const QuestArgs& a);
+
+// Stochastic index selection: the draw from the rest of each row (stochastic.cu).
+constexpr int kMaxSelectScratch = 64;   // ints of block-scan and selection state
+struct SampleArgs {
+    const int32_t* lens;
+    const int32_t* k_det;
+    const int32_t* k_samp;
+    int32_t* idx;            // in: the exact top-k_det rows; out: those rows and the drawn ones
+    int32_t* status;
+    uint64_t seed;
+    uint32_t step;
+    int B, Hq, k_max;
+    long n_cap;
+    int words;               // 32-bit words of a bitmap over n_cap positions
+    int cap;                 // candidate positions that fit in shared memory
+};
+size_t sample_smem(const SampleArgs& a);
+cudaError_t launch_sample(const SampleArgs& a, cudaStream_t stream);
 
 struct AppendArgs {
     __nv_bfloat16* K;

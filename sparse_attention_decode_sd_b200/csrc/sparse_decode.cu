@@ -280,6 +280,7 @@ __global__ void __launch_bounds__(1024, 2) rows_kernel(DecodeArgs a) {
     const int r = blockIdx.x * a.rpc + rl;
     const int k_max = a.k_max;
     int first_neg = k_max;
+    int drawn = 0;   // weighted mode: entries carrying kSampledFlag
     if (r < R) {   // uniform over the row's warps
         const int b = r / a.Hq;
         const int n = checked_len(a.lens, b, a.n_cap, a.status);
@@ -289,7 +290,16 @@ __global__ void __launch_bounds__(1024, 2) rows_kernel(DecodeArgs a) {
             int v[kRowBatch];
 #pragma unroll
             for (int i = 0; i < kRowBatch; ++i) v[i] = j0 + i < k_max ? __ldg(row + j0 + i) : -1;
-            const int pv = (lane == 0 && j0 > 0) ? __ldg(row + j0 - 1) : -1;
+            int pv = (lane == 0 && j0 > 0) ? __ldg(row + j0 - 1) : -1;
+            if (a.weighted) {   // positions without the flag; count the drawn entries
+#pragma unroll
+                for (int i = 0; i < kRowBatch; ++i)
+                    if (v[i] >= 0) {
+                        drawn += (v[i] & kSampledFlag) ? 1 : 0;
+                        v[i] &= kPosMask;
+                    }
+                if (pv >= 0) pv &= kPosMask;
+            }
             int p = __shfl_up_sync(0xffffffffu, v[kRowBatch - 1], 1);
             if (lane == 0) p = pv;
 #pragma unroll
@@ -309,14 +319,26 @@ __global__ void __launch_bounds__(1024, 2) rows_kernel(DecodeArgs a) {
         }
     }
     first_neg = __reduce_min_sync(0xffffffffu, first_neg);
-    if (lane == 0) s_neg[warp] = first_neg;
+    drawn = __reduce_add_sync(0xffffffffu, drawn);
+    __shared__ int s_drawn[32];
+    if (lane == 0) {
+        s_neg[warp] = first_neg;
+        s_drawn[warp] = drawn;
+    }
     __syncthreads();
     if (t == 0) {
-        int m = k_max;
-        for (int w = 0; w < wpr; ++w) m = min(m, s_neg[rl * wpr + w]);
+        int m = k_max, dr = 0;
+        for (int w = 0; w < wpr; ++w) {
+            m = min(m, s_neg[rl * wpr + w]);
+            dr += s_drawn[rl * wpr + w];
+        }
         if (r < R) {
             a.rlen[r] = m;
             a.arrive[r] = 0;
+            if (a.weighted) {   // each drawn entry stands for (N_b - plain entries) / drawn rows
+                const int n = checked_len(a.lens, r / a.Hq, a.n_cap, nullptr);
+                a.rlw[r] = dr > 0 && n > m - dr ? log2f((float)(n - (m - dr)) / (float)dr) : 0.f;
+            }
         } else {
             m = 0;
         }
@@ -344,7 +366,8 @@ constexpr int kGatherTile = 4 * kHalfBlock;                 // K and V, both hal
 struct SparseSmem {   // placed at a 1024-byte aligned address (swizzle atoms)
     uint8_t kv[kSparseStages][kGatherTile];
     uint64_t full[kSparseStages];           // TMA completion of each stage
-    int info[kSparseStages][4];             // rows | flags << 5 | valid-row mask << 16, row, segment slot, segments
+    int info[kSparseStages][4];             // rows | flags << 5 | valid-row mask << 16, row,
+                                            // segment slot | segments << 16, drawn-row mask
     uint32_t q[kSparseStages][kHeadDim / 2];   // q of the row a tile opens (bf16 pairs)
 };
 
@@ -434,7 +457,8 @@ __device__ __forceinline__ RowTile next_row_tile(const DecodeArgs& a, RowWalker&
 // inside the page-table row (below max_pages * 16) are looked up.
 __device__ __forceinline__ void lookup_pages(const DecodeArgs& a, RowTile& d) {
     const int lane = threadIdx.x & 31;
-    if (d.v >= 0 && d.v < a.n_cap) d.page = __ldcg(a.page_table + d.pt_off + (d.v >> 4));
+    const int pos = a.weighted ? (d.v & kPosMask) : d.v;
+    if (d.v >= 0 && pos < a.n_cap) d.page = __ldcg(a.page_table + d.pt_off + (pos >> 4));
     if ((d.hdr >> 5) & kFlagFirst) d.q2 = __ldcg(reinterpret_cast<const uint2*>(a.q + (long)d.r * kHeadDim) + lane);
 }
 
@@ -465,14 +489,16 @@ __device__ __forceinline__ void issue_row_tile(const DecodeArgs& a, SparseSmem& 
         if (d.page >= 0 && d.page < a.num_pages) {
             ok = true;
             ri = ((uint32_t)d.page * kPageSize + (uint32_t)(d.v & (kPageSize - 1))) * (uint32_t)a.Hkv + (uint32_t)d.kvh;
+            // (the flag bit of a drawn entry lies above the slot bits used here)
         } else {
             report(a.status, SD_ERR_INDEX_OOB);   // a page entry outside the cache, or a position at or past N_b
         }
     }
     const uint32_t okm = __ballot_sync(0xffffffffu, ok);
+    const uint32_t drawn = a.weighted ? __ballot_sync(0xffffffffu, ok && (d.v & kSampledFlag)) : 0u;
     if (lane == 0)
-        *reinterpret_cast<int4*>(ws.info[st]) = make_int4((d.hdr & 0xff) | (int)((okm & 0xffffu) << 16), d.r,
-                                                          d.seg & 0xffff, d.seg >> 16);
+        *reinterpret_cast<int4*>(ws.info[st]) =
+            make_int4((d.hdr & 0xff) | (int)((okm & 0xffffu) << 16), d.r, d.seg, (int)(drawn & 0xffffu));
     if ((d.hdr >> 5) & kFlagFirst) reinterpret_cast<uint2*>(ws.q[st])[lane] = d.q2;
     if (rows == 0) return;
     const uint32_t sub = okm ? __shfl_sync(0xffffffffu, ri, __ffs(okm) - 1) : 0u;   // every lane takes part
@@ -501,6 +527,7 @@ __device__ __forceinline__ void issue_row_tile(const DecodeArgs& a, SparseSmem& 
 // and column 1 their bf16 residual, so the head's output is the sum of accumulator columns 0 and 1
 // (lanes with lane % 4 == 0 hold both).
 struct HeadState {
+    float lw;           // weighted mode: log2 of the weight of the row's drawn entries
     float m;            // running max of column 0 (log2 units; lanes % 4 == 0)
     float l;            // partial sum of rows g, g + 8 (lanes % 4 == 0)
     float acc[8][4];    // O^T fragments: dims 16 mt + g (+ 8) x columns 2 (lane % 4) (+ 1)
@@ -508,7 +535,7 @@ struct HeadState {
 };
 
 __device__ __forceinline__ void reset_head(HeadState& st) {
-    st.m = -INFINITY;
+    st.m = -INFINITY;   // (lw belongs to the row and is set when its first tile is consumed)
     st.l = 0.f;
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) st.acc[mt][0] = st.acc[mt][1] = st.acc[mt][2] = st.acc[mt][3] = 0.f;
@@ -526,7 +553,7 @@ __device__ __forceinline__ void load_q_head(const uint32_t* qr, HeadState& st) {
 
 // One tile: S = K_tile . q (8 MMAs), masked online softmax over the tile's valid rows, O^T += V_tile^T .
 // [p_hi, p_lo] (8 MMAs).  `koff` / `voff` are this lane's ldmatrix offsets (row and chunk, swizzled).
-__device__ __forceinline__ void compute_row_tile(const DecodeArgs& a, uint32_t tile, uint32_t valid,
+__device__ __forceinline__ void compute_row_tile(const DecodeArgs& a, uint32_t tile, uint32_t valid, uint32_t drawn,
                                                  const uint32_t (&koff)[4], const uint32_t (&voff)[4],
                                                  HeadState& st) {
     const int lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
@@ -539,8 +566,12 @@ __device__ __forceinline__ void compute_row_tile(const DecodeArgs& a, uint32_t t
         else mma_bf16_16816(s, a0, a1, a2, a3, st.qb[j][0], st.qb[j][1]);
     }
     // column 0: rows g (s[0]) and g + 8 (s[2]) in lanes with c == 0
-    const float z0 = ((valid >> g) & 1u) ? (s[0] + s2[0]) * a.scale_log2 : -INFINITY;
-    const float z1 = ((valid >> (g + 8)) & 1u) ? (s[2] + s2[2]) * a.scale_log2 : -INFINITY;
+    // (a drawn entry's logit is raised by log2 of its weight: its exp is multiplied by the weight)
+    const float z0 = ((valid >> g) & 1u) ? (s[0] + s2[0]) * a.scale_log2 + (((drawn >> g) & 1u) ? st.lw : 0.f)
+                                         : -INFINITY;
+    const float z1 = ((valid >> (g + 8)) & 1u)
+                         ? (s[2] + s2[2]) * a.scale_log2 + (((drawn >> (g + 8)) & 1u) ? st.lw : 0.f)
+                         : -INFINITY;
     float tm = fmaxf(z0, z1);
     tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 4));
     tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, 8));
@@ -823,6 +854,7 @@ __global__ void __launch_bounds__(32) sparse_decode_kernel(DecodeArgs a, const _
     static_assert(kSparseStages == 2, "the pipeline gathers one tile ahead");
     HeadState st;
     reset_head(st);
+    st.lw = 0.f;
     bool ok = true;
     for (;; ++t) {
         const int stage = t & (kSparseStages - 1);
@@ -839,13 +871,17 @@ __global__ void __launch_bounds__(32) sparse_decode_kernel(DecodeArgs a, const _
         const int4 info = *reinterpret_cast<const int4*>(ws.info[stage]);
         const int flags = (info.x >> 5) & 7;
         if (flags & kFlagEnd) break;
-        if (flags & kFlagFirst) load_q_head(ws.q[stage], st);
+        if (flags & kFlagFirst) {
+            load_q_head(ws.q[stage], st);
+            st.lw = a.weighted ? __ldcg(a.rlw + info.y) : 0.f;
+        }
         ok = mbar_wait(&ws.full[stage], (uint32_t)((t / kSparseStages) & 1));
         ok = __all_sync(0xffffffffu, ok);   // warp-uniform before the collective ops below
         if (!ok) break;
-        compute_row_tile(a, kv0 + (uint32_t)(stage * kGatherTile), (uint32_t)info.x >> 16, koff, voff, st);
+        compute_row_tile(a, kv0 + (uint32_t)(stage * kGatherTile), (uint32_t)info.x >> 16, (uint32_t)info.w, koff,
+                         voff, st);
         if (flags & kFlagLast) {
-            finish_row_segment(a, info.y, info.z, info.w, st);
+            finish_row_segment(a, info.y, info.z & 0xffff, info.z >> 16, st);
             reset_head(st);
         }
         __syncwarp();   // every lane has read the stage before it is refilled

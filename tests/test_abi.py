@@ -74,11 +74,11 @@ def test_workspace_sizes(lib):
     small = rows * 8192 * 8 + rows * 4 + 3 * 8             # (head, page) records, thresholds, pointers
     assert scores + small <= topk <= scores + small + 4 * 256
     # sparse decode: 64 segment partials per (b, h) row (fp32 output + max and sum), per row its
-    # length and arrival counter, then one length sum per CTA of the row pass (1 row per CTA at
-    # k_max 2621)
+    # length and arrival counter, one length sum per CTA of the row pass (1 row per CTA at k_max
+    # 2621), and per row the weight of drawn rows (stochastic selection)
     sparse = sdb.sd_workspace_size(s, sdb.SD_OP_SPARSE)
-    need = rows * 64 * (128 * 4 + 8) + rows * 4 * 2 + rows * 4
-    assert need <= sparse <= need + 5 * 256
+    need = rows * 64 * (128 * 4 + 8) + rows * 4 * 2 + rows * 4 + rows * 4
+    assert need <= sparse <= need + 6 * 256
     # dense decode: min(N, 1280) + 1 segment partials per (b, h) and one row count per 16384 positions
     # of every (b, KV head) group
     dense = sdb.sd_workspace_size(s, sdb.SD_OP_DENSE)
