@@ -148,7 +148,40 @@ SparseLayout sparse_layout(const Dims& d) {
 }
 // entries of all rows are counted in int32
 bool sparse_fits(const Dims& d) { return (long)d.B * d.Hq * d.k_max < (1L << 31); }
-size_t decode_workspace(const Dims& d, bool dense) { return dense ? dense_layout(d).total : sparse_layout(d).total; }
+
+// The sparse decode walks GQA groups (one gathered row serves every head of the group that selected
+// it) instead of heads when the shape says the heads' selections overlap heavily: with a fraction
+// f = k_max / capacity selected per head, independent selections of the G heads would have the
+// group read G f N rows per head walk against (1 - (1 - f)^G) N rows of their union.
+constexpr double kUnionDuplication = 1.4;
+bool use_group_walk(const Dims& d) {
+    const double f = d.n_cap > 0 ? (double)d.k_max / (double)d.n_cap : 1.0;
+    const double fc = f < 1.0 ? f : 1.0;
+    const double uni = 1.0 - pow(1.0 - fc, (double)d.G);
+    return uni > 0.0 && d.G * fc / uni >= kUnionDuplication;
+}
+
+// sparse decode over GQA groups: the row pass's part of the sparse layout, then the dense layout,
+// then the groups' selection masks [B*Hkv][n_cap] (1 byte per position for G <= 8, else 2)
+struct UnionLayout {
+    SparseLayout rows;
+    DenseLayout grp;
+    size_t base_grp, umask, total;
+};
+UnionLayout union_layout(const Dims& d) {
+    UnionLayout L;
+    L.rows = sparse_layout(d);
+    L.grp = dense_layout(d);
+    L.base_grp = L.rows.total;
+    L.umask = L.base_grp + L.grp.total;
+    L.total = L.umask + align256((size_t)d.B * d.Hkv * d.n_cap * (d.G <= 8 ? 1 : 2));
+    return L;
+}
+
+size_t decode_workspace(const Dims& d, bool dense) {
+    if (dense) return dense_layout(d).total;
+    return use_group_walk(d) ? union_layout(d).total : sparse_layout(d).total;
+}
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -211,6 +244,26 @@ sd_status decode_common(const sd_shape* shape, const void* q, const void* K, con
         a.counts = reinterpret_cast<int*>(ws + L.counts);
         a.jmax = d.jmax;
         return launch_status(launch_dense(a, s));
+    }
+    if (use_group_walk(d) && !weighted) {   // (drawn rows are weighted by the per-head walk, whose
+                                             // workspace lies at the start of this layout)
+        const UnionLayout U = union_layout(d);
+        a.rlen = reinterpret_cast<int*>(ws + U.rows.rlen);
+        a.arrive = reinterpret_cast<int*>(ws + U.rows.arrive);
+        a.bsum = reinterpret_cast<int*>(ws + U.rows.bsum);
+        a.rlw = reinterpret_cast<float*>(ws + U.rows.rlw);
+        a.tpr = U.rows.tpr;
+        a.rpc = U.rows.rpc;
+        a.nb = U.rows.nb;
+        a.weighted = weighted ? 1 : 0;
+        a.acc = reinterpret_cast<float*>(ws + U.base_grp + U.grp.acc);
+        a.ml = reinterpret_cast<float2*>(ws + U.base_grp + U.grp.ml);
+        a.counts = reinterpret_cast<int*>(ws + U.base_grp + U.grp.counts);
+        a.umask = ws + U.umask;
+        a.jmax = d.jmax;
+        int gw = di.sms * di.decode_ctas_per_sm[1][d.G > 8 ? 1 : 0];
+        a.total_warps = gw > kMaxDecodeWarps ? kMaxDecodeWarps : gw;
+        return launch_status(launch_sparse_union(a, s));
     }
     const SparseLayout L = sparse_layout(d);
     a.acc = reinterpret_cast<float*>(ws + L.acc);

@@ -65,8 +65,10 @@ struct DecodeArgs {
     int* arrive;          // [B*Hq] segments of the row finished so far (zeroed by rows_kernel)
     int* bsum;            // [nb] entries of the rows of each rows_kernel CTA
     float* rlw;           // [B*Hq] weighted mode: log2 of the weight of the row's drawn entries
-    // workspace, dense decode
-    int* counts;          // [nrt] rows per range
+    // workspace, dense decode and the sparse decode over GQA groups
+    int* counts;          // [nrt] rows (positions) per range
+    uint8_t* umask;       // sparse over groups: [B*Hkv][n_cap] heads of the group that selected each
+                          // position (bit g: head kvh*G+g), 1 byte per position for G <= 8, else 2
     // workspace, both
     float2* ml;           // per (b, h, segment) running max (log2 units) and sum
     float* acc;           // per (b, h, segment) un-normalised output [128]
@@ -89,6 +91,7 @@ size_t sparse_decode_smem();
 // CTAs (one warp each) of the decode kernel for (dense, G) that fit on one SM.
 cudaError_t decode_occupancy(bool dense, int G, int* ctas_per_sm);
 cudaError_t launch_sparse(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_sparse_union(const DecodeArgs& a, cudaStream_t stream);
 cudaError_t launch_dense(const DecodeArgs& a, cudaStream_t stream);
 
 // Quest page-level indexer.

@@ -26,7 +26,9 @@ std::mutex g_static_mu;
 void* g_static_ptr[kMaxDevices] = {};
 
 // Device address of the scratch on the current device, looked up once per device (with that
-// device current) on its first call.
+// device current) on its first call and kept.  The address belongs to the device's context: after
+// a cudaDeviceReset the library's device code is loaded again, so the entry point must not be
+// called after a reset in the same process (documented in the header).
 sd_status static_scratch(void** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return SD_ERR_CUDA;

@@ -37,6 +37,7 @@
 #include <cudaTypedefs.h>
 
 #include <mutex>
+#include <type_traits>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -912,6 +913,85 @@ __global__ void __launch_bounds__(256) ranges_kernel(DecodeArgs a) {
     a.counts[ri] = lo < n ? min(kRange, n - lo) : 0;
 }
 
+// ---------------------------------------------------------------------------------------------
+// sparse decode over GQA groups: union_masks_kernel
+// ---------------------------------------------------------------------------------------------
+// First index j of an idx row (ascending positions, then negative padding) whose position is at
+// least `target` (len if none): a 32-way search by one warp, every probe of a round in flight
+// together.  Negative entries count as past every position.
+__device__ __forceinline__ int first_at_least(const int32_t* row, int len, int target) {
+    const int lane = threadIdx.x & 31;
+    int lo = 0, hi = len;   // the answer lies in [lo, hi]
+    while (hi - lo > 32) {
+        const int step = (hi - lo + 31) / 32;
+        const int x = min(lo + (lane + 1) * step - 1, hi - 1);
+        const int v = __ldg(row + x);
+        const uint32_t ge = __ballot_sync(0xffffffffu, v < 0 || v >= target);
+        if (ge == 0u) {
+            lo = min(lo + 32 * step, hi);   // past the last probe (which is hi - 1)
+        } else {
+            const int f = __ffs(ge) - 1;
+            const int xf = min(lo + (f + 1) * step - 1, hi - 1);
+            lo = f == 0 ? lo : min(lo + f * step, hi);
+            hi = xf;
+        }
+    }
+    const int x = lo + lane;
+    const int v = x < hi ? __ldg(row + x) : 0;
+    const uint32_t ge = __ballot_sync(0xffffffffu, x < hi && (v < 0 || v >= target));
+    return ge ? lo + __ffs(ge) - 1 : hi;
+}
+
+// One CTA per (group, kRange-position range): the heads of the group that selected each position,
+// as bits of a per-position mask (MT: 8 bits for G <= 8, 16 for G <= 16) in the workspace, and the
+// range's position count (the unit the group walk is split in).  Each warp finds a head's entries
+// in the range by a 32-way search of its idx row and sets their bits in shared memory.
+template <typename MT>
+__global__ void __launch_bounds__(256) union_masks_kernel(DecodeArgs a) {
+    constexpr int kPer = 4 / (int)sizeof(MT);            // masks per 32-bit word
+    __shared__ uint32_t m[kRange / kPer];
+    pdl_enter();
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int ri = blockIdx.x;
+    const int grp = ri / a.nrp, rloc = ri - grp * a.nrp;
+    const int b = grp / a.Hkv, kvh = grp - b * a.Hkv;
+    const int n = checked_len(a.lens, b, a.n_cap, a.status);
+    const int r0 = rloc * kRange, r1 = min(n, r0 + kRange);
+    if (tid == 0) a.counts[ri] = r1 > r0 ? r1 - r0 : 0;
+    if (r0 >= r1) return;
+    for (int i = tid; i < kRange / kPer; i += blockDim.x) m[i] = 0u;
+    __syncthreads();
+    for (int g = warp; g < a.G; g += (int)(blockDim.x >> 5)) {
+        const int32_t* row = a.idx + ((long)b * a.Hq + (long)kvh * a.G + g) * a.k_max;
+        const int lo = first_at_least(row, a.k_max, r0);
+        const int hi = first_at_least(row, a.k_max, r1);
+        if (hi - lo == r1 - r0) {
+            // every position of the range (strictly ascending entries in [r0, r1)): the head's bit in
+            // every mask, one word per lane
+            uint32_t rep = 0u;
+#pragma unroll
+            for (int i = 0; i < kPer; ++i) rep |= (1u << g) << (8 * (int)sizeof(MT) * i);
+            const int words = (r1 - r0 + kPer - 1) / kPer;
+            for (int i = lane; i < words; i += 32) {
+                const int pl = (i + 1) * kPer - (r1 - r0);   // positions of the last word past r1
+                atomicOr(&m[i], pl > 0 ? rep & (0xffffffffu >> (8 * (int)sizeof(MT) * pl)) : rep);
+            }
+            continue;
+        }
+        for (int j = lo + lane; j < hi; j += 32) {
+            const int p = __ldg(row + j) - r0;
+            if (p >= 0 && p < r1 - r0)   // (an unsorted row is reported by rows_kernel)
+                atomicOr(&m[p / kPer], (1u << g) << (8 * (int)sizeof(MT) * (p % kPer)));
+        }
+    }
+    __syncthreads();
+    // positions r0 .. r1 - 1 of the group's masks (rounded up to 16 bytes: still inside the group's
+    // row, whose length max_pages * 16 is a multiple of 16)
+    uint4* dst = reinterpret_cast<uint4*>(a.umask + ((long)grp * a.n_cap + r0) * (long)sizeof(MT));
+    const int nvec = ((r1 - r0) * (int)sizeof(MT) + 15) / 16;
+    for (int i = tid; i < nvec; i += blockDim.x) dst[i] = reinterpret_cast<const uint4*>(m)[i];
+}
+
 // The warp's walk over its rows (all fields warp-uniform).
 struct GroupWalker {
     int e, e_end;     // next global row and the end of this warp's share
@@ -921,6 +1001,10 @@ struct GroupWalker {
     int seg_j;        // segment slot of the current segment
     bool seg_new;     // the next tile opens a segment
     int epw;          // rows per warp
+    // group walk over selected positions: this lane's head mask in the 32-position window (aligned
+    // within range ri) at offset win, and in the window after it, loaded one window ahead
+    int win, nwin;    // window offsets in range ri (-1: none)
+    uint32_t wmk, nmk;
 };
 
 // The next non-empty range after ri (one exists while rows remain; at the last range *cnt = 0).
@@ -934,6 +1018,10 @@ __device__ __forceinline__ int next_range(const DecodeArgs& a, int ri, int* cnt)
     return ri;
 }
 
+// The next tile of a group walk.  Dense: the next 16 positions, every head.  Union (kUnion): the
+// walk still advances over positions, but a tile takes only the positions some head of the group
+// selected (mask != 0, 32 positions examined per round), each with its heads' mask.
+template <int NT, bool kUnion>
 __device__ __forceinline__ TileDesc prefetch_group_tile(const DecodeArgs& a, GroupWalker& w) {
     const int lane = threadIdx.x & 31;
     TileDesc d = empty_tile();
@@ -957,6 +1045,53 @@ __device__ __forceinline__ TileDesc prefetch_group_tile(const DecodeArgs& a, Gro
             w.ri = ri;
             w.off = 0;
             w.cnt = c;
+            w.win = w.nwin = -1;
+        }
+        if (kUnion) {
+            using MT = typename std::conditional<NT == 1, uint8_t, uint16_t>::type;
+            const MT* gm = reinterpret_cast<const MT*>(a.umask) + (long)grp * a.n_cap +
+                           (long)(w.ri - grp * a.nrp) * kRange;   // the masks of range ri
+            const int wo = w.off & ~31;
+            if (w.win != wo) {   // enter the window: from the prefetch, else loaded now
+                w.wmk = (w.nwin == wo) ? w.nmk : (wo + lane < w.cnt ? (uint32_t)__ldg(gm + wo + lane) : 0u);
+                w.win = wo;
+                w.nwin = wo + 32 < w.cnt ? wo + 32 : -1;
+                w.nmk = (w.nwin >= 0 && w.nwin + lane < w.cnt) ? (uint32_t)__ldg(gm + w.nwin + lane) : 0u;
+            }
+            // positions w.off .. limit - 1 of this window are examined
+            const int limit = min(min(wo + 32, w.cnt), w.off + (w.e_end - w.e));
+            if (limit <= w.off) {   // not reached (counts are consistent); ends the walk
+                w.e = w.e_end;
+                break;
+            }
+            const int at = wo + lane;
+            uint32_t take = __ballot_sync(0xffffffffu, at >= w.off && at < limit && w.wmk != 0u);
+            int consumed = limit - w.off;
+            const int need = kTileRows - filled;
+            if (__popc(take) > need) {   // the tile fills up: stop after the need-th selected position
+                const int last = (int)__fns(take, 0, need);
+                take &= last == 31 ? 0xffffffffu : ((2u << last) - 1u);
+                consumed = wo + last + 1 - w.off;
+            }
+            const int cnt = __popc(take);
+            const bool mine = lane >= filled && lane < filled + cnt;
+            const int src = mine ? (int)__fns(take, 0, lane - filled + 1) : 0;
+            const uint32_t msrc = __shfl_sync(0xffffffffu, w.wmk, src);
+            if (mine) {
+                const int p = (w.ri - grp * a.nrp) * kRange + wo + src;
+                const int page = __ldg(a.page_table + (long)b * a.max_pages + p / kPageSize);
+                if (page < 0 || page >= a.num_pages) {
+                    report(a.status, SD_ERR_INDEX_OOB);
+                    d.row_idx = kNoRow;
+                } else {
+                    d.row_idx = ((uint32_t)page * kPageSize + (uint32_t)(p & (kPageSize - 1))) * (uint32_t)a.Hkv + kvh;
+                }
+                d.mask = msrc;
+            }
+            filled += cnt;
+            w.off += consumed;
+            w.e += consumed;
+            continue;
         }
         const int take = min(min(kTileRows - filled, w.cnt - w.off), w.e_end - w.e);
         if (take <= 0) {   // not reached (counts are consistent); ends the walk
@@ -990,6 +1125,7 @@ __device__ __forceinline__ TileDesc prefetch_group_tile(const DecodeArgs& a, Gro
             w.ri = ri;   // the next segment starts in range ri
             w.off = 0;
             w.cnt = c;
+            w.win = w.nwin = -1;
             w.grp = ri / a.nrp;
             w.seg_j = (int)(blockIdx.x - w.e / w.epw);   // w.e is the first row of the new group
             w.seg_new = true;
@@ -1059,7 +1195,7 @@ __device__ __forceinline__ int sum_counts(const DecodeArgs& a, int lo, int hi) {
     return __reduce_add_sync(0xffffffffu, s);
 }
 
-template <int NT>
+template <int NT, bool kUnion>
 __global__ void __launch_bounds__(32) dense_decode_kernel(DecodeArgs a) {
     extern __shared__ __align__(128) uint8_t smem[];
     DecodeSmem& ws = *reinterpret_cast<DecodeSmem*>(smem);
@@ -1103,23 +1239,25 @@ __global__ void __launch_bounds__(32) dense_decode_kernel(DecodeArgs a) {
     w.off = w.e - ri0;
     w.cnt = __ldg(a.counts + ri);
     w.grp = ri / a.nrp;
+    w.win = w.nwin = -1;
+    w.wmk = w.nmk = 0u;
     const int e0grp = ri0 - sum_counts(a, w.grp * a.nrp, ri);   // first row of the group
     w.seg_j = (int)(blockIdx.x - e0grp / w.epw);
     w.seg_new = true;
 
     Softmax<NT> st;
     reset_state(st);
-    TileDesc next = prefetch_group_tile(a, w);
+    TileDesc next = prefetch_group_tile<NT, kUnion>(a, w);
 #pragma unroll
     for (int s = 0; s < kStages - 1; ++s) {
         issue_tile(a, ws, s, next);
-        next = prefetch_group_tile(a, w);
+        next = prefetch_group_tile<NT, kUnion>(a, w);
     }
     for (int t = 0;; ++t) {
         const int stage = t % kStages;
         // the stage of tile t-1 is free: issue tile t+kStages-1 before waiting for tile t
         issue_tile(a, ws, (t + kStages - 1) % kStages, next);
-        next = prefetch_group_tile(a, w);
+        next = prefetch_group_tile<NT, kUnion>(a, w);
         cp_async_wait<kStages - 1>();
         __syncwarp();
         const int rows = ws.info[stage][0], flags = ws.info[stage][1];
@@ -1254,7 +1392,15 @@ cudaError_t decode_occupancy(bool dense, int G, int* ctas_per_sm) {
         if (e != cudaSuccess) return e;
         return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, sparse_decode_kernel, 32, smem);
     }
-    return G <= 8 ? occupancy_of(dense_decode_kernel<1>, ctas_per_sm) : occupancy_of(dense_decode_kernel<2>, ctas_per_sm);
+    // (the group walk over selected positions runs with the same shared memory and occupancy)
+    int union_ctas = 0;
+    cudaError_t e = G <= 8 ? occupancy_of(dense_decode_kernel<1, true>, &union_ctas)
+                           : occupancy_of(dense_decode_kernel<2, true>, &union_ctas);
+    if (e != cudaSuccess) return e;
+    e = G <= 8 ? occupancy_of(dense_decode_kernel<1, false>, ctas_per_sm)
+               : occupancy_of(dense_decode_kernel<2, false>, ctas_per_sm);
+    if (e == cudaSuccess && union_ctas < *ctas_per_sm) *ctas_per_sm = union_ctas;
+    return e;
 }
 
 namespace {
@@ -1325,12 +1471,28 @@ cudaError_t launch_sparse(const DecodeArgs& a, cudaStream_t stream) {
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
+// Sparse decode over GQA groups (rows many heads of a group share): row checks, the groups'
+// selection masks, the group walk over the selected positions, the merge of the segments.
+cudaError_t launch_sparse_union(const DecodeArgs& a, cudaStream_t stream) {
+    cudaError_t e = launch_pdl(rows_kernel, dim3(a.nb), dim3(a.tpr * a.rpc), 0, stream, a);
+    if (e != cudaSuccess) return e;
+    e = a.G <= 8 ? launch_pdl(union_masks_kernel<uint8_t>, dim3((unsigned)a.nrt), dim3(256), 0, stream, a)
+                 : launch_pdl(union_masks_kernel<uint16_t>, dim3((unsigned)a.nrt), dim3(256), 0, stream, a);
+    if (e != cudaSuccess) return e;
+    const dim3 grid(a.total_warps), block(32);
+    e = a.G <= 8 ? launch_pdl(dense_decode_kernel<1, true>, grid, block, decode_smem(), stream, a)
+                 : launch_pdl(dense_decode_kernel<2, true>, grid, block, decode_smem(), stream, a);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(merge_kernel, dim3((unsigned)((long)a.B * a.Hq)), dim3(kMergeWarps * 32), 0, stream, a);
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
 cudaError_t launch_dense(const DecodeArgs& a, cudaStream_t stream) {
     cudaError_t e = launch_pdl(ranges_kernel, dim3((unsigned)((a.nrt + 255) / 256)), dim3(256), 0, stream, a);
     if (e != cudaSuccess) return e;
     const dim3 grid(a.total_warps), block(32);
-    e = a.G <= 8 ? launch_pdl(dense_decode_kernel<1>, grid, block, decode_smem(), stream, a)
-                 : launch_pdl(dense_decode_kernel<2>, grid, block, decode_smem(), stream, a);
+    e = a.G <= 8 ? launch_pdl(dense_decode_kernel<1, false>, grid, block, decode_smem(), stream, a)
+                 : launch_pdl(dense_decode_kernel<2, false>, grid, block, decode_smem(), stream, a);
     if (e != cudaSuccess) return e;
     e = launch_pdl(merge_kernel, dim3((unsigned)((long)a.B * a.Hq)), dim3(kMergeWarps * 32), 0, stream, a);
     return e != cudaSuccess ? e : cudaGetLastError();

@@ -280,6 +280,16 @@ __global__ void __launch_bounds__(kSelectThreads, 2) select_kernel(TopkArgs a) {
         select_masked(src, take, row, hist, scratch, s_sel);
     }
     for (int i = take + tid; i < a.k_max; i += nthr) row[i] = -1;
+    // The row's records are dead now: their L2 lines are dropped without being written back (only
+    // lines that lie wholly inside this row's records), so that they cost no DRAM write bandwidth
+    // in the kernels that follow.  The next score pass rewrites every record it reads.
+    __syncthreads();
+    {
+        const uintptr_t lo = reinterpret_cast<uintptr_t>(src.rec), hi = lo + (uintptr_t)src.np * sizeof(uint2);
+        const uintptr_t first = (lo + 127) & ~(uintptr_t)127, end = hi & ~(uintptr_t)127;
+        for (uintptr_t ad = first + (uintptr_t)tid * 128; ad < end; ad += (uintptr_t)nthr * 128)
+            asm volatile("discard.global.L2 [%0], 128;" ::"l"(ad) : "memory");
+    }
 }
 
 // ---------------------------------------------------------------------------------------------

@@ -121,6 +121,41 @@ def test_decode_repeated_calls_reuse_the_workspace():
         gh.check_outputs(out.cpu().numpy(), ref)
 
 
+GROUP_WALK = [
+    # B, Hq, Hkv, lens, k_max, per-head fraction selected: heads of a group that share most rows
+    # make the decode walk groups (one gathered row serves every head that selected it)
+    (2, 16, 4, [20000, 7000], 12000, 0.6),    # two 16384-position ranges, ragged
+    (1, 32, 2, [40000], 30000, 0.7),          # G = 16 (16-bit head masks)
+    (3, 8, 2, [50000, 0, 333], 25000, 0.5),   # an empty request and a short one
+    (2, 8, 4, [17000, 16384], 16384, 1.0),    # G = 2, k = N: every row, range edges
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,lens,k_max,frac", GROUP_WALK)
+def test_group_walk_arbitrary_rows(B, Hq, Hkv, lens, k_max, frac):
+    """Per-head random subsets of a large fraction of the rows (some heads empty, one with a single
+    row), decoded through the group walk, against the oracle on the same rows."""
+    w_cpu = wl.make_workload(B, Hq, Hkv, lens, 1, seed=sum(lens) + Hq, k_max=k_max)
+    g = torch.Generator().manual_seed(B * 1000 + Hq)
+    idx = torch.full((B, Hq, k_max), -1, dtype=torch.int32)
+    for b in range(B):
+        n = int(w_cpu.lens[b])
+        for h in range(Hq):
+            cnt = min(k_max, n, int(frac * n))
+            if h == 1:
+                cnt = 0
+            elif h == 2:
+                cnt = min(1, n)
+            idx[b, h, :cnt] = torch.randperm(n, generator=g)[:cnt].sort().values.to(torch.int32)
+    w = w_cpu.to(DEV)
+    r = gh.Runner(w)
+    out = r.sparse(idx.to(DEV))
+    assert r.device_status() == 0
+    ref = oracle.attend(w_cpu.shape(), w_cpu.q, w_cpu.K, w_cpu.V, w_cpu.page_table, w_cpu.lens, idx)
+    gh.check_outputs(out.cpu().numpy(), ref)
+    assert (out[:, 1] == 0).all()
+
+
 @pytest.mark.parametrize("n,k", [(3000, 100), (40000, 100), (40000, 39999)])
 def test_exact_ties_go_to_lower_positions(n, k):
     """Identical K rows: every score ties, so the selection is exactly positions 0..k-1.  With N

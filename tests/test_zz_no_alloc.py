@@ -3,9 +3,10 @@ handed only its inputs and outputs, a service with a fixed device-memory plan). 
 workspace (score rows, candidate counts) in a 48 MiB array inside the library instead of a caller
 workspace.
 
-Checked through the C ABI against sd_topk_index with an ordinary workspace, on two calls in a row
-with different shapes (the second call reuses the array the first one filled), and the size limit
-is rejected before any launch.  This file is collected last on purpose."""
+Checked through the C ABI against sd_topk_index with an ordinary workspace, on calls in a row with
+different shapes in both orders (a small call after a large one reuses an array whose candidate
+records and thresholds the large call left behind, and the reverse), and the size limit is rejected
+before any launch.  This file is collected last on purpose."""
 from __future__ import annotations
 
 import ctypes
@@ -40,9 +41,10 @@ def _both(w):
 
 
 def test_static_scratch_matches_workspace_version_twice():
-    first = wl.make_workload(2, 16, 4, [9000, 5000], [180, 100], seed=41, device="cuda")
-    second = wl.make_workload(1, 64, 8, 131072, 2621, seed=42, structure="sinks3", device="cuda")   # just over 32 MiB
-    for w in (first, second):
+    small = wl.make_workload(2, 16, 4, [9000, 5000], [180, 100], seed=41, device="cuda")
+    # one long-context request: about 33 MiB of the 48 MiB array
+    large = wl.make_workload(1, 64, 8, 131072, 2621, seed=42, structure="sinks3", device="cuda")
+    for w in (small, large, small, large):
         ref, got = _both(w)
         assert torch.equal(ref, got)   # integer output: identical
 
