@@ -42,8 +42,8 @@ L2_FLUSH_BYTES = 512 << 20
 NOMINAL_HBM_GBS = 8000.0   # HBM3e, nominal (context for the effective-bandwidth fractions)
 # kernels of one step: threshold, score pass, select; rows, sparse decode
 LAUNCHES_PER_STEP = 5
-# kernels of one Quest step: last-page box refresh, page score, page select; rows, sparse decode
-QUEST_LAUNCHES_PER_STEP = 5
+# kernels of one Quest step: page score, page select; rows, sparse decode
+QUEST_LAUNCHES_PER_STEP = 4
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -366,7 +366,9 @@ def quest_k_max(w) -> int:
 
 
 def time_quest(w, flush, stream, steps: int, warmup: int):
-    """Quest step: last-page box refresh + page index (the index leg), then sparse decode."""
+    """Quest step: page index (the index leg), then sparse decode.  The page boxes are kept current by
+    the append of each step (sd_quest_append_kv: the written page's box updated in the same pass), so
+    the step itself reads them as they are; here K does not change between steps."""
     dev = w.q.device
     k_max = quest_k_max(w)
     shape = sdb.make_shape(w.B, w.Hq, w.Hkv, w.max_pages, k_max, w.num_pages)
@@ -379,7 +381,6 @@ def time_quest(w, flush, stream, steps: int, warmup: int):
     sdb.sd_quest_summarize(shape, w.K, w.page_table, w.lens, boxes, status, stream=stream)   # the prefill's part
 
     def index():
-        sdb.sd_quest_summarize(shape, w.K, w.page_table, w.lens, boxes, status, last_page_only=True, stream=stream)
         sdb.sd_quest_index(shape, w.q, boxes, w.page_table, w.lens, w.k, idx, ws_q, status, stream)
 
     def decode():
@@ -712,8 +713,8 @@ def run_ours(args):
 
 
 def run_quest(args):
-    """The step with the Quest page-level indexer in place of the exact one: refresh each request's
-    last page box (what a decode loop does after appending), select pages, sparse decode."""
+    """The step with the Quest page-level indexer in place of the exact one: select pages from the
+    page boxes (kept current by the append of a decode loop, sd_quest_append_kv), sparse decode."""
     world, rank, local = dist_setup()
     dev = torch.device("cuda", local)
     kw = {"ratio": args.ratio} if args.workload == "sweep128k" else {}

@@ -223,6 +223,16 @@ SD_API sd_status sd_quest_summarize(const sd_shape* shape, const void* K, const 
                                     const int32_t* lens, void* boxes, int32_t last_page_only,
                                     int32_t* dev_status, void* stream);
 
+/* sd_append_kv that also keeps the Quest boxes current: the box of the page each row is written to
+ * becomes the row itself when the row opens the page (p % 16 == 0), else the elementwise min / max of
+ * the stored box and the row -- the same bf16 values sd_quest_summarize would write for the page's
+ * rows, without a separate pass over K after each step.  Same arguments, checks and errors as
+ * sd_append_kv, plus boxes (as for sd_quest_summarize; NULL or misaligned: SD_ERR_INVALID_ARG).  The
+ * boxes of the other pages must be current already (sd_quest_summarize over the whole cache once). */
+SD_API sd_status sd_quest_append_kv(const sd_shape* shape, void* K, void* V, const int32_t* page_table,
+                                    int32_t* lens, const void* k_new, const void* v_new, int32_t* k_sel,
+                                    int32_t ratio, void* boxes, int32_t* dev_status, void* stream);
+
 /* sd_quest_index selects, per (b, h), ceil(k[b] / 16) pages: the current page (holding position
  * N_b - 1) plus the most relevant others, relevance of page j being the largest q.k any key inside its
  * box can reach, r_j = sum_d max(q_d * min_d, q_d * max_d) (fp32 accumulation of exact bf16 products);

@@ -33,7 +33,7 @@ SD_SAMPLED_FLAG = 1 << 30   # idx entry of a row drawn by sd_stochastic_index (p
 
 EXPORTED = ("sd_workspace_size", "sd_topk_index", "sd_topk_scores", "sd_topk_select", "sd_topk_index_static",
             "sd_sparse_decode", "sd_stochastic_index", "sd_sparse_decode_sampled", "sd_dense_decode", "sd_append_kv",
-            "sd_quest_summarize", "sd_quest_index", "sd_selftest_wait_timeout", "sd_status_string",
+            "sd_quest_summarize", "sd_quest_append_kv", "sd_quest_index", "sd_selftest_wait_timeout", "sd_status_string",
             "sd_last_cuda_error", "sd_version")
 
 
@@ -79,13 +79,14 @@ def load():
     lib.sd_stochastic_index.argtypes = [SH, P, P, P, P, P, P, ctypes.c_uint64, ctypes.c_uint32, P, P, SZ, P, P]
     lib.sd_dense_decode.argtypes = [SH, P, P, P, P, P, P, P, SZ, P, P]
     lib.sd_append_kv.argtypes = [SH, P, P, P, P, P, P, P, I32, P, P]
+    lib.sd_quest_append_kv.argtypes = [SH, P, P, P, P, P, P, P, I32, P, P, P]
     lib.sd_quest_summarize.argtypes = [SH, P, P, P, P, I32, P, P]
     lib.sd_quest_index.argtypes = [SH, P, P, P, P, P, P, P, SZ, P, P]
     lib.sd_selftest_wait_timeout.argtypes = [ctypes.c_uint32, P, P]
     lib.sd_selftest_wait_timeout.restype = I32
     for f in (lib.sd_workspace_size, lib.sd_topk_index, lib.sd_topk_scores, lib.sd_topk_select, lib.sd_sparse_decode,
               lib.sd_sparse_decode_sampled, lib.sd_stochastic_index, lib.sd_dense_decode, lib.sd_append_kv,
-              lib.sd_quest_summarize, lib.sd_quest_index):
+              lib.sd_quest_summarize, lib.sd_quest_append_kv, lib.sd_quest_index):
         f.restype = I32
     lib.sd_status_string.argtypes = [I32]
     lib.sd_status_string.restype = ctypes.c_char_p
@@ -240,6 +241,15 @@ def sd_append_kv(shape, K, V, page_table, lens, k_new, v_new, k_sel, ratio, dev_
     st = load().sd_append_kv(ctypes.byref(shape), _ptr(K), _ptr(V), _ptr(page_table), _ptr(lens), _ptr(k_new),
                              _ptr(v_new), _ptr(k_sel), int(ratio), _ptr(dev_status), _stream(stream))
     return _check(st, "sd_append_kv", check)
+
+
+def sd_quest_append_kv(shape, K, V, page_table, lens, k_new, v_new, k_sel, ratio, boxes, dev_status, stream=None,
+                       check=True) -> int:
+    """sd_append_kv that also brings the Quest box of each written page up to date."""
+    st = load().sd_quest_append_kv(ctypes.byref(shape), _ptr(K), _ptr(V), _ptr(page_table), _ptr(lens), _ptr(k_new),
+                                   _ptr(v_new), _ptr(k_sel), int(ratio), _ptr(boxes), _ptr(dev_status),
+                                   _stream(stream))
+    return _check(st, "sd_quest_append_kv", check)
 
 
 def workspace_for(shape: SdShape, op: int, device=None) -> torch.Tensor:

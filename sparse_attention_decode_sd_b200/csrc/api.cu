@@ -153,13 +153,23 @@ bool sparse_fits(const Dims& d) { return (long)d.B * d.Hq * d.k_max < (1L << 31)
 // it) instead of heads when the shape says the heads' selections overlap heavily: with a fraction
 // f = k_max / capacity selected per head, independent selections of the G heads would have the
 // group read G f N rows per head walk against (1 - (1 - f)^G) N rows of their union.
-constexpr double kUnionDuplication = 1.4;
-bool use_group_walk(const Dims& d) {
+// Expected duplication of a GQA group's selections: entries per distinct position when each head
+// selects a fraction f = k_max / capacity of the positions independently, G f / (1 - (1 - f)^G).
+double expected_duplication(const Dims& d) {
     const double f = d.n_cap > 0 ? (double)d.k_max / (double)d.n_cap : 1.0;
     const double fc = f < 1.0 ? f : 1.0;
     const double uni = 1.0 - pow(1.0 - fc, (double)d.G);
-    return uni > 0.0 && d.G * fc / uni >= kUnionDuplication;
+    return uni > 0.0 ? d.G * fc / uni : 1.0;
 }
+constexpr double kUnionDuplication = 1.4;   // from here on, one gathered tile serves a group's heads
+constexpr double kOrderDuplication = 1.1;   // from here on, the per-head walk aligns a group's heads
+bool use_group_walk(const Dims& d) { return expected_duplication(d) >= kUnionDuplication; }
+// Expected fraction of a group's positions that some head selects: 1 - (1 - f)^G.
+double expected_coverage(const Dims& d) {
+    const double f = d.n_cap > 0 ? (double)d.k_max / (double)d.n_cap : 1.0;
+    return 1.0 - pow(1.0 - (f < 1.0 ? f : 1.0), (double)d.G);
+}
+constexpr double kUnionTilesCoverage = 0.9;   // from here on, the group walk takes whole tiles
 
 // sparse decode over GQA groups: the row pass's part of the sparse layout, then the dense layout,
 // then the groups' selection masks [B*Hkv][n_cap] (1 byte per position for G <= 8, else 2)
@@ -261,6 +271,7 @@ sd_status decode_common(const sd_shape* shape, const void* q, const void* K, con
         a.counts = reinterpret_cast<int*>(ws + U.base_grp + U.grp.counts);
         a.umask = ws + U.umask;
         a.jmax = d.jmax;
+        a.union_tiles = expected_coverage(d) >= kUnionTilesCoverage ? 1 : 0;
         int gw = di.sms * di.decode_ctas_per_sm[1][d.G > 8 ? 1 : 0];
         a.total_warps = gw > kMaxDecodeWarps ? kMaxDecodeWarps : gw;
         return launch_status(launch_sparse_union(a, s));
@@ -277,6 +288,7 @@ sd_status decode_common(const sd_shape* shape, const void* q, const void* K, con
     a.rpc = L.rpc;
     a.nb = L.nb;
     a.jmax = kRowSegs;
+    a.order_rows = (d.G > 1 && (long)d.B * d.Hq <= kOrderMaxRows && expected_duplication(d) >= kOrderDuplication) ? 1 : 0;
     a.min_epw = (d.k_max + kRowSegs - 2) / (kRowSegs - 1);   // ceil(k_max / (kRowSegs - 1))
     return launch_status(launch_sparse(a, s));
 }
@@ -467,9 +479,10 @@ sd_status sd_dense_decode(const sd_shape* shape, const void* q, const void* K, c
                          stream, true);
 }
 
-sd_status sd_append_kv(const sd_shape* shape, void* K, void* V, const int32_t* page_table, int32_t* lens,
-                       const void* k_new, const void* v_new, int32_t* k_sel, int32_t ratio, int32_t* dev_status,
-                       void* stream) {
+namespace {
+sd_status append_common(const sd_shape* shape, void* K, void* V, const int32_t* page_table, int32_t* lens,
+                        const void* k_new, const void* v_new, int32_t* k_sel, int32_t ratio, void* boxes,
+                        int32_t* dev_status, void* stream) {
     Dims d;
     sd_status st = check_shape(shape, &d);
     if (st != SD_OK) return st;
@@ -485,6 +498,7 @@ sd_status sd_append_kv(const sd_shape* shape, void* K, void* V, const int32_t* p
     a.k_new = static_cast<const __nv_bfloat16*>(k_new);
     a.v_new = static_cast<const __nv_bfloat16*>(v_new);
     a.k_sel = k_sel;
+    a.boxes = static_cast<__nv_bfloat16*>(boxes);
     a.status = dev_status;
     a.B = d.B;
     a.Hkv = d.Hkv;
@@ -492,6 +506,20 @@ sd_status sd_append_kv(const sd_shape* shape, void* K, void* V, const int32_t* p
     a.num_pages = d.num_pages;
     a.ratio = ratio;
     return launch_status(launch_append(a, static_cast<cudaStream_t>(stream)));
+}
+}  // namespace
+
+sd_status sd_append_kv(const sd_shape* shape, void* K, void* V, const int32_t* page_table, int32_t* lens,
+                       const void* k_new, const void* v_new, int32_t* k_sel, int32_t ratio, int32_t* dev_status,
+                       void* stream) {
+    return append_common(shape, K, V, page_table, lens, k_new, v_new, k_sel, ratio, nullptr, dev_status, stream);
+}
+
+sd_status sd_quest_append_kv(const sd_shape* shape, void* K, void* V, const int32_t* page_table, int32_t* lens,
+                             const void* k_new, const void* v_new, int32_t* k_sel, int32_t ratio, void* boxes,
+                             int32_t* dev_status, void* stream) {
+    if (boxes == nullptr || !aligned(boxes, 16)) return SD_ERR_INVALID_ARG;
+    return append_common(shape, K, V, page_table, lens, k_new, v_new, k_sel, ratio, boxes, dev_status, stream);
 }
 
 namespace {

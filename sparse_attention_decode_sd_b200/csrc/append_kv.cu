@@ -1,5 +1,9 @@
 // append_kv.cu -- one decode step's K/V row per request written into its page (the growing cache
-// of an agentic decode loop), plus the length and per-request k that the next step uses.
+// of an agentic decode loop), plus the length and per-request k that the next step uses.  With Quest
+// boxes ("The Sparse Frontier" review, sec. 7.1: per page and KV head the per-dimension minimum and
+// maximum of its keys) the box of the written page is brought up to date in the same pass: the new
+// key row alone when it opens the page, else the elementwise min / max with the stored box (min and
+// max are associative, so the result equals a summary of the page's rows).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -29,12 +33,38 @@ __global__ void __launch_bounds__(128) append_kernel(AppendArgs a) {
     }
     __syncthreads();
     if (!s_ok) return;
+    const bool opens_page = (a.lens[b] % kPageSize) == 0;   // read before the length is advanced below
     for (int i = threadIdx.x; i < a.Hkv * 16; i += blockDim.x) {
         const int kvh = i >> 4, ch = i & 15;
         const long dst = (s_row + kvh) * kHeadDim + ch * 8;
         const long src = ((long)b * a.Hkv + kvh) * kHeadDim + ch * 8;
-        *reinterpret_cast<uint4*>(a.K + dst) = *reinterpret_cast<const uint4*>(a.k_new + src);
+        const uint4 kr = *reinterpret_cast<const uint4*>(a.k_new + src);
+        *reinterpret_cast<uint4*>(a.K + dst) = kr;
         *reinterpret_cast<uint4*>(a.V + dst) = *reinterpret_cast<const uint4*>(a.v_new + src);
+        if (a.boxes != nullptr) {
+            const long page = s_row / ((long)kPageSize * a.Hkv);
+            uint4* bmin = reinterpret_cast<uint4*>(a.boxes + ((page * a.Hkv + kvh) * 2) * kHeadDim + ch * 8);
+            uint4* bmax = reinterpret_cast<uint4*>(a.boxes + ((page * a.Hkv + kvh) * 2 + 1) * kHeadDim + ch * 8);
+            if (opens_page) {
+                *bmin = kr;
+                *bmax = kr;
+            } else {
+                uint4 lo = *bmin, hi = *bmax;
+                uint32_t* l = reinterpret_cast<uint32_t*>(&lo);
+                uint32_t* h = reinterpret_cast<uint32_t*>(&hi);
+                const uint32_t* k = reinterpret_cast<const uint32_t*>(&kr);
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {   // bf16 pairs: min and max are exact
+                    const __nv_bfloat162 kv = *reinterpret_cast<const __nv_bfloat162*>(&k[t]);
+                    const __nv_bfloat162 mn = __hmin2(*reinterpret_cast<const __nv_bfloat162*>(&l[t]), kv);
+                    const __nv_bfloat162 mx = __hmax2(*reinterpret_cast<const __nv_bfloat162*>(&h[t]), kv);
+                    l[t] = *reinterpret_cast<const uint32_t*>(&mn);
+                    h[t] = *reinterpret_cast<const uint32_t*>(&mx);
+                }
+                *bmin = lo;
+                *bmax = hi;
+            }
+        }
     }
     __syncthreads();
     if (threadIdx.x == 0) {

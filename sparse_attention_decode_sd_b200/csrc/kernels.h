@@ -48,6 +48,7 @@ constexpr int kRange = 16384;           // dense decode: positions per counted r
 constexpr int kMaxDecodeWarps = 1280;   // dense decode: persistent warps (one per CTA) at most
 constexpr int kMaxSparseWarps = 4096;   // sparse decode: persistent warps (one per CTA) at most
 constexpr int kRowSegs = 64;            // sparse decode: segment slots per (b, h) row
+constexpr int kOrderMaxRows = 2048;     // sparse decode: rows up to which the offset order is used
 constexpr int kRowBatch = 4;            // sparse decode: consecutive idx entries per rows_kernel thread and pass
 constexpr uint32_t kSampledFlag = 0x40000000u;   // idx entry: a row drawn by the stochastic selection
 constexpr int kPosMask = 0x3fffffff;             // the position bits of an idx entry
@@ -84,6 +85,9 @@ struct DecodeArgs {
     float scale_log2;     // log2(e) / sqrt(d)
     int weighted;         // sparse: idx entries with kSampledFlag are drawn rows of a stochastic
                           // selection, weighted by (N_b - plain entries) / drawn entries
+    int order_rows;       // sparse: full rows are visited in offset order (heads of a group aligned)
+    int union_tiles;      // group walk: whole 16-position tiles with head masks, instead of only the
+                          // selected positions (the union covers nearly every position)
 };
 
 size_t decode_smem();
@@ -142,6 +146,7 @@ struct AppendArgs {
     const __nv_bfloat16* k_new;
     const __nv_bfloat16* v_new;
     int32_t* k_sel;
+    __nv_bfloat16* boxes;   // Quest boxes [num_pages][Hkv][2][128] kept up to date for the written page, or null
     int32_t* status;
     int B, Hkv, max_pages, num_pages, ratio;
 };

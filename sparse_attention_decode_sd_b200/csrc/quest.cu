@@ -176,6 +176,7 @@ __global__ void __launch_bounds__(256) quest_score_kernel(QuestArgs a, long unit
 // select: one CTA per (b, h)
 // ---------------------------------------------------------------------------------------------
 constexpr int kQuestSelectThreads = 512;
+constexpr int kQuestLoads = 16;   // relevance loads in flight per thread (8192 pages per round)
 
 // Keys of the pages 0 .. n - 1 in shared memory; an element's position is its page index.
 struct PageKeys {
@@ -220,11 +221,33 @@ __global__ void __launch_bounds__(kQuestSelectThreads) quest_select_kernel(Quest
         for (int i = tid; i < a.k_max; i += nthr) row[i] = (i < n) ? i : -1;
         return;
     }
-    // the kp - 1 most relevant pages among 0 .. np - 2 (np - 1, the current page, is always kept)
+    // the kp - 1 most relevant pages among 0 .. np - 2 (np - 1, the current page, is always kept):
+    // their keys, kQuestLoads relevance loads in flight per thread, and the keys' range
     const float* rrow = a.rel + bh * a.max_pages;
-    for (int j = tid; j < np - 1; j += nthr) lkey[j] = float_key(rrow[j]);
+    reset_key_range(s_sel);
     __syncthreads();
-    if (kp > 1) select_exact(PageKeys{lkey, np - 1}, kp - 1, kept, hist, scratch, s_sel);
+    uint32_t kmin = 0xffffffffu, kmax = 0u;
+    for (int j0 = tid; j0 < np - 1; j0 += kQuestLoads * nthr) {
+        float v[kQuestLoads];
+#pragma unroll
+        for (int u = 0; u < kQuestLoads; ++u) {
+            const int j = j0 + u * nthr;
+            v[u] = j < np - 1 ? __ldcg(rrow + j) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < kQuestLoads; ++u) {
+            const int j = j0 + u * nthr;
+            if (j < np - 1) {
+                const uint32_t key = float_key(v[u]);
+                lkey[j] = key;
+                kmin = min(kmin, key);
+                kmax = max(kmax, key);
+            }
+        }
+    }
+    add_key_range(s_sel, kmin, kmax);
+    __syncthreads();
+    if (kp > 1) select_exact(PageKeys{lkey, np - 1}, kp - 1, kept, hist, scratch, s_sel, true);
     __syncthreads();
     // positions of the kept pages, ascending: kp - 1 full pages, then the (possibly partial) current page
     for (int i = tid; i < a.k_max; i += nthr) {

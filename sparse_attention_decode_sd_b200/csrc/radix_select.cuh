@@ -56,33 +56,45 @@ __device__ __forceinline__ void select_bin(const int* hist, int nbins, int targe
 // ranked directly by one warp instead of running the next digit's histogram.
 constexpr int kSmallBin = 64;
 
-template <class Visit>
-__device__ void radix_select(Visit visit, int target, int* hist, int* scratch, int* s_sel, uint32_t* T_out,
-                             int* greater_out) {
-    const int tid = threadIdx.x, nthr = blockDim.x, lane = tid & 31;
-    uint32_t kmin = 0xffffffffu, kmax = 0u;
-    visit([&](uint32_t key) {
-        kmin = min(kmin, key);
-        kmax = max(kmax, key);
-    });
+// The block's key range, for a caller that writes the keys: reset_key_range before the pass (and a
+// barrier), add_key_range with each thread's (min, max) after it, then a barrier; key_range reads it.
+__device__ __forceinline__ void reset_key_range(int* s_sel) {
+    if (threadIdx.x == 0) {
+        reinterpret_cast<unsigned int*>(s_sel)[2] = 0xffffffffu;
+        reinterpret_cast<unsigned int*>(s_sel)[3] = 0u;
+    }
+}
+__device__ __forceinline__ void add_key_range(int* s_sel, uint32_t kmin, uint32_t kmax) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
         kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
         kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
     }
+    if ((threadIdx.x & 31) == 0) {
+        atomicMin(reinterpret_cast<unsigned int*>(s_sel) + 2, kmin);
+        atomicMax(reinterpret_cast<unsigned int*>(s_sel) + 3, kmax);
+    }
+}
+
+// have_range: the caller filled the key range (reset_key_range / add_key_range and a barrier).
+template <class Visit>
+__device__ void radix_select(Visit visit, int target, int* hist, int* scratch, int* s_sel, uint32_t* T_out,
+                             int* greater_out, bool have_range = false) {
+    const int tid = threadIdx.x, nthr = blockDim.x, lane = tid & 31;
     unsigned int* range = reinterpret_cast<unsigned int*>(s_sel + 2);
-    if (tid == 0) {
-        range[0] = 0xffffffffu;
-        range[1] = 0u;
+    if (!have_range) {
+        uint32_t kmin = 0xffffffffu, kmax = 0u;
+        visit([&](uint32_t key) {
+            kmin = min(kmin, key);
+            kmax = max(kmax, key);
+        });
+        reset_key_range(s_sel);
+        __syncthreads();
+        add_key_range(s_sel, kmin, kmax);
+        __syncthreads();
     }
-    __syncthreads();
-    if (lane == 0) {
-        atomicMin(&range[0], kmin);
-        atomicMax(&range[1], kmax);
-    }
-    __syncthreads();
-    kmin = range[0];
-    kmax = range[1];
+    uint32_t kmin = range[0];
+    uint32_t kmax = range[1];
     __syncthreads();
     const uint32_t diff = kmin ^ kmax;
     int top = diff ? 31 - __clz(diff) : -1;   // highest bit that differs; above it every key is kmin's
@@ -155,13 +167,13 @@ __device__ void radix_select(Visit visit, int target, int* hist, int* scratch, i
 
 template <class Src>
 __device__ __forceinline__ void radix_find(const Src& src, int target, int* hist, int* scratch, int* s_sel,
-                                           uint32_t* T_out, int* greater_out) {
+                                           uint32_t* T_out, int* greater_out, bool have_range) {
     const int n = src.size();
     radix_select(
         [&](auto f) {
             for (int j = threadIdx.x; j < n; j += blockDim.x) f(src.key(j));
         },
-        target, hist, scratch, s_sel, T_out, greater_out);
+        target, hist, scratch, s_sel, T_out, greater_out, have_range);
 }
 
 // Writes the selected positions of src in ascending order to row[0..take): keys above T, plus the
@@ -194,10 +206,11 @@ __device__ void emit_selected(const Src& src, uint32_t T, int quota, int take, i
 }
 
 template <class Src>
-__device__ void select_exact(const Src& src, int take, int32_t* row, int* hist, int* scratch, int* s_sel) {
+__device__ void select_exact(const Src& src, int take, int32_t* row, int* hist, int* scratch, int* s_sel,
+                             bool have_range = false) {
     uint32_t T;
     int greater;
-    radix_find(src, take, hist, scratch, s_sel, &T, &greater);
+    radix_find(src, take, hist, scratch, s_sel, &T, &greater, have_range);
     emit_selected(src, T, take - greater, take, row, scratch);
 }
 

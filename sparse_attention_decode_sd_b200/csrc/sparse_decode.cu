@@ -3,30 +3,41 @@
 // survey sec. 1.1 restricted to the selected set), and the dense comparator over every row
 // ("Dense" mode of the same figure).
 //
-// Sparse decode, two kernels per call:
+// Sparse decode, two kernels per call (per-head walk):
 //   rows_kernel           one group of threads per (request, query head) row of idx: checks the row
 //                         (ascending positions below N_b, then negative padding only), finds its length
 //                         (the index of the first negative entry), zeroes the output of empty rows and
-//                         the row's arrival counter, and writes per-CTA length sums.
+//                         the row's arrival counter, and writes per-CTA length sums.  Rows of a
+//                         stochastic selection (weighted mode) also get the log2 weight of their drawn
+//                         entries.  It releases the decode grid as soon as it starts.
 //   sparse_decode_kernel  one warp per CTA, a persistent grid of one wave (12 warps per SM).  The
-//                         selected entries of all rows, in (request, head, position) order, are cut
-//                         evenly across the warps; a warp finds its first row from the length sums and
-//                         streams its entries in tiles of 16 rows.  Per tile, in a software pipeline
-//                         that waits for no load but the gather itself: the positions are loaded four
-//                         tiles ahead, mapped through the page table two tiles ahead, and the 256-byte
-//                         K and V rows gathered one tile ahead by TMA four-row gathers (tile::gather4,
-//                         64-dim halves with the 128-byte swizzle) into a two-stage shared-memory ring.
-//                         The heads of a GQA group are consecutive rows, so their warps run side by side
-//                         and a row several of them selected is mostly served from L2 after its first
-//                         read.  On the tensor cores (mma.sync m16n8k16, bf16 in, fp32 accumulate):
+//                         selected entries of all rows are cut evenly across the warps and each warp
+//                         streams its entries in tiles of 16 rows.  The walk starts before rows_kernel
+//                         ends, on the split that holds when every row has k_max entries (the
+//                         indexer's rows); after the wait, the entry count confirms that split or the
+//                         walk restarts on the row lengths.  Full rows are visited in the order of
+//                         their start offset inside a warp's share, so that the G heads of a GQA
+//                         group read the positions they share at the same time (the second read comes
+//                         from L2).  Per tile, in a software pipeline that waits for no load but the
+//                         gather itself: positions loaded four tiles ahead, mapped through the page
+//                         table two tiles ahead, and the 256-byte K and V rows gathered one tile ahead
+//                         by TMA four-row gathers (tile::gather4, 64-dim halves with the 128-byte
+//                         swizzle) into a two-stage shared-memory ring.  On the tensor cores
+//                         (mma.sync m16n8k16, bf16 in, fp32 accumulate):
 //                             S   = K_tile (16 rows x 128) . q              8 MMAs (q: column 0 of B)
 //                             o  += V_tile^T (128 x 16 rows) . [p_hi, p_lo] 8 MMAs (columns 0 and 1 of B)
 //                         with an fp32 online softmax in between; the weights p enter as a bf16 high
 //                         part and a bf16 residual, and the head's output is the sum of the two
-//                         accumulator columns.  A warp's part of one row is a "segment": a row held by
-//                         one warp is written out directly; otherwise each warp stores its (max, sum,
-//                         output) partial and the last of the row's warps to arrive (a counter per
-//                         row) merges the partials by log-sum-exp.
+//                         accumulator columns.  A warp's part of one row is a "segment": each warp
+//                         stores its (max, sum, output) partial and the last of the row's warps to
+//                         arrive (a counter per row) merges the partials by log-sum-exp; a row held
+//                         by one warp is written out directly.
+//
+// Sparse decode over GQA groups (chosen by the host when the heads of a group are expected to
+// share many rows), four kernels: rows_kernel as above; union_masks_kernel sets, per (group,
+// 16384-position range), a byte (two for G > 8) per position whose bits are the heads that selected
+// it; dense_decode_kernel<., true> walks only the masked positions of every group, one gathered tile
+// serving every head that selected its rows; merge_kernel combines the partials.
 //
 // Dense decode (the comparator), three kernels: ranges_kernel counts the positions of each
 // kRange-position range of every (request, KV head) group; dense_decode_kernel walks all rows of every
@@ -266,7 +277,10 @@ __device__ __forceinline__ int warp_inclusive_scan(int v) {
 // its length (the index of the first negative entry), zeroes the output of empty rows and the
 // row's arrival counter, and writes per-CTA length sums.  Positions are mapped to cache rows by the
 // decode kernel itself, as it streams.
-__global__ void __launch_bounds__(1024, 2) rows_kernel(DecodeArgs a) {
+// U passes over a row have their loads in flight together (rows longer than two passes take U = 4,
+// with one CTA per SM for the registers).
+template <int U>
+__global__ void __launch_bounds__(1024, U == 1 ? 2 : 1) rows_kernel(DecodeArgs a) {
     __shared__ int s_neg[32];   // per warp: first negative entry it saw
     __shared__ int s_len[32];   // per row of this CTA
     // The decode kernel is released only after this wait: when its grid starts, all earlier work in
@@ -286,36 +300,44 @@ __global__ void __launch_bounds__(1024, 2) rows_kernel(DecodeArgs a) {
         const int b = r / a.Hq;
         const int n = checked_len(a.lens, b, a.n_cap, a.status);
         const int32_t* row = a.idx + (long)r * k_max;
-        for (int base = 0; base < k_max; base += tpr * kRowBatch) {   // uniform over the row's threads
-            const int j0 = base + t * kRowBatch;
-            int v[kRowBatch];
+        for (int base = 0; base < k_max; base += U * tpr * kRowBatch) {   // uniform over the row's threads
+            int v[U][kRowBatch], pv[U];
 #pragma unroll
-            for (int i = 0; i < kRowBatch; ++i) v[i] = j0 + i < k_max ? __ldg(row + j0 + i) : -1;
-            int pv = (lane == 0 && j0 > 0) ? __ldg(row + j0 - 1) : -1;
-            if (a.weighted) {   // positions without the flag; count the drawn entries
+            for (int u = 0; u < U; ++u) {   // pass u: entries base + u tpr kRowBatch + ...
+                const int j0 = base + (u * tpr + t) * kRowBatch;
 #pragma unroll
-                for (int i = 0; i < kRowBatch; ++i)
-                    if (v[i] >= 0) {
-                        drawn += (v[i] & kSampledFlag) ? 1 : 0;
-                        v[i] &= kPosMask;
-                    }
-                if (pv >= 0) pv &= kPosMask;
+                for (int i = 0; i < kRowBatch; ++i) v[u][i] = j0 + i < k_max ? __ldg(row + j0 + i) : -1;
+                // the entry before this warp's first one (inside the row)
+                pv[u] = (lane == 0 && j0 > 0 && j0 < k_max) ? __ldg(row + j0 - 1) : -1;
             }
-            int p = __shfl_up_sync(0xffffffffu, v[kRowBatch - 1], 1);
-            if (lane == 0) p = pv;
 #pragma unroll
-            for (int i = 0; i < kRowBatch; ++i) {
-                const int j = j0 + i;
-                if (j < k_max) {
-                    if (v[i] < 0) {
-                        first_neg = min(first_neg, j);
-                    } else if (v[i] >= n) {
-                        report(a.status, SD_ERR_INDEX_OOB);
-                    } else if (j > 0 && (p < 0 || p >= v[i])) {
-                        report(a.status, SD_ERR_ORDER);
-                    }
+            for (int u = 0; u < U; ++u) {
+                const int j0 = base + (u * tpr + t) * kRowBatch;
+                if (a.weighted) {   // positions without the flag; count the drawn entries
+#pragma unroll
+                    for (int i = 0; i < kRowBatch; ++i)
+                        if (v[u][i] >= 0) {
+                            drawn += (v[u][i] & kSampledFlag) ? 1 : 0;
+                            v[u][i] &= kPosMask;
+                        }
+                    if (pv[u] >= 0) pv[u] &= kPosMask;
                 }
-                p = v[i];
+                int p = __shfl_up_sync(0xffffffffu, v[u][kRowBatch - 1], 1);
+                if (lane == 0) p = pv[u];
+#pragma unroll
+                for (int i = 0; i < kRowBatch; ++i) {
+                    const int j = j0 + i;
+                    if (j < k_max) {
+                        if (v[u][i] < 0) {
+                            first_neg = min(first_neg, j);
+                        } else if (v[u][i] >= n) {
+                            report(a.status, SD_ERR_INDEX_OOB);
+                        } else if (j > 0 && (p < 0 || p >= v[u][i])) {
+                            report(a.status, SD_ERR_ORDER);
+                        }
+                    }
+                    p = v[u][i];
+                }
             }
         }
     }
@@ -389,7 +411,31 @@ struct RowWalker {
     bool full;           // every row holds k_max entries (row lengths need no lookup)
     bool seg_new;        // the next tile opens a segment
     int seq;             // tiles handed out so far
+    int o_lane, o_step;  // offset order: o(lane) and 32 k_max mod epw
 };
+
+// With full rows, the walk's slot i (entries [i k_max, (i + 1) k_max)) starts at offset
+// o(i) = i k_max mod epw inside a warp's share, and every warp advances through its share at about
+// the same pace: the entry at offset o is reached at about the same time o / rate in every warp.
+// Rows are given to slots in the order of (o(i), i), so the G heads of a GQA group sit in slots of
+// nearly equal offset and read the positions they share at nearly the same time: the second read
+// comes from L2.  (In plain row order sibling heads drift apart by k_max mod epw per row.)  Row of
+// slot i = the rank of (o(i), i) among all slots, counted by the warp (R / 32 steps per lane).
+template <bool kOrder>
+__device__ __forceinline__ int row_of_slot(const DecodeArgs& a, const RowWalker& w, int slot) {
+    if constexpr (!kOrder) return slot;
+    const int lane = threadIdx.x & 31;
+    const int R = a.B * a.Hq;
+    const int o = (int)((uint32_t)(slot * a.k_max) % (uint32_t)w.epw);   // slot k_max < 2^31
+    int oi = w.o_lane;
+    int rank = 0;
+    for (int i = lane; i < R; i += 32) {
+        rank += (oi < o || (oi == o && i < slot)) ? 1 : 0;
+        oi += w.o_step;
+        if (oi >= w.epw) oi -= w.epw;
+    }
+    return __reduce_add_sync(0xffffffffu, rank);
+}
 
 __device__ __forceinline__ void enter_row(const DecodeArgs& a, RowWalker& w, int r, int rstart, int len) {
     const int R = a.B * a.Hq;
@@ -418,6 +464,7 @@ struct RowTile {
 };
 
 // The next tile of the walk; issues the loads of its positions (first used two steps later).
+template <bool kOrder>
 __device__ __forceinline__ RowTile next_row_tile(const DecodeArgs& a, RowWalker& w) {
     const int lane = threadIdx.x & 31;
     RowTile d;
@@ -442,11 +489,15 @@ __device__ __forceinline__ RowTile next_row_tile(const DecodeArgs& a, RowWalker&
     if (w.e == w.rend || w.e == w.e_end) {
         flags |= kFlagLast;
         if (w.e < w.e_end) {   // the next non-empty row (one exists: entries remain)
-            const int R = a.B * a.Hq;
-            int r = w.r + 1;
-            int len = w.next_len;
-            while (len == 0 && r + 1 < R) len = __ldg(a.rlen + (++r));
-            enter_row(a, w, r, w.rend, len);
+            if (kOrder && w.full) {   // the next slot's row
+                enter_row(a, w, row_of_slot<kOrder>(a, w, w.rend / a.k_max), w.rend, a.k_max);
+            } else {
+                const int R = a.B * a.Hq;
+                int r = w.r + 1;
+                int len = w.next_len;
+                while (len == 0 && r + 1 < R) len = __ldg(a.rlen + (++r));
+                enter_row(a, w, r, w.rend, len);
+            }
         }
     }
     d.hdr = rows | (flags << 5) | (stage << 8);
@@ -695,6 +746,7 @@ __device__ __forceinline__ void finish_row_segment(const DecodeArgs& a, int r, i
     merge_row(a, r, nseg);
 }
 
+template <bool kOrder>
 __global__ void __launch_bounds__(32) sparse_decode_kernel(DecodeArgs a, const __grid_constant__ CUtensorMap kmap,
                                                            const __grid_constant__ CUtensorMap vmap) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -727,14 +779,14 @@ __global__ void __launch_bounds__(32) sparse_decode_kernel(DecodeArgs a, const _
     const uint32_t kv0 = smem_addr(ws.kv);
     RowTile dA, dB, dC;   // the pipeline's tile records (see the main loop)
     auto start_pipeline = [&]() {
-        dA = next_row_tile(a, w);
-        dB = next_row_tile(a, w);
-        dC = next_row_tile(a, w);
+        dA = next_row_tile<kOrder>(a, w);
+        dB = next_row_tile<kOrder>(a, w);
+        dC = next_row_tile<kOrder>(a, w);
         lookup_pages(a, dA);
         issue_row_tile(a, ws, kv0, dA, &kmap, &vmap);   // the walk's first tile
         dA = dB;
         dB = dC;
-        dC = next_row_tile(a, w);
+        dC = next_row_tile<kOrder>(a, w);
         lookup_pages(a, dA);
     };
     // Speculative start on the split that holds when every row has k_max entries (the indexer's
@@ -744,27 +796,42 @@ __global__ void __launch_bounds__(32) sparse_decode_kernel(DecodeArgs a, const _
     const long e_full = (long)R * a.k_max;   // < 2^31 (checked on the host)
     w.full = true;
     w.epw = max(a.min_epw, (int)((e_full + a.total_warps - 1) / a.total_warps));
+    if (kOrder) {
+        w.o_lane = (int)((uint64_t)lane * (uint64_t)a.k_max % (uint64_t)w.epw);
+        w.o_step = (int)(32ull * (uint64_t)a.k_max % (uint64_t)w.epw);
+    }
     const bool spec = (long)blockIdx.x * w.epw < e_full;
     if (spec) {
         w.e = (int)blockIdx.x * w.epw;
         w.e_end = (int)min(e_full, (long)w.e + w.epw);
-        const int r = w.e / a.k_max;
-        enter_row(a, w, r, r * a.k_max, a.k_max);
+        const int slot = w.e / a.k_max;
+        enter_row(a, w, row_of_slot<kOrder>(a, w, slot), slot * a.k_max, a.k_max);
         start_pipeline();
     }
-    pdl_wait();   // rows_kernel: row lengths, checks, zeroed arrival counters
-    // E = all entries: the length sums of the rows_kernel CTAs, each lane summing kPrologue
-    // consecutive ones per round
+    // The row pass's results -- row checks, lengths, zeroed arrival counters, drawn-row weights -- are
+    // needed before this warp's first global write (a segment's partial or a row's output) and before
+    // any read of them.  A warp on the full-row split waits only then (at its first segment end),
+    // with its first tiles already consumed; the entry count E = R * k_max confirms its split, else
+    // the tiles in flight are drained and the walk restarts on the row lengths.  Weighted mode reads
+    // the drawn-row weights when a row opens, so it waits before the loop.
     int E = 0;
-    for (int base = 0; base < a.nb; base += 32 * kPrologue) {
-        const int k0 = base + kPrologue * lane;
+    bool confirmed = false;
+    auto wait_rows = [&]() {
+        pdl_wait();
+        // E = all entries: the length sums of the rows_kernel CTAs, each lane summing kPrologue
+        // consecutive ones per round
+        int sum = 0;
+        for (int base = 0; base < a.nb; base += 32 * kPrologue) {
+            const int k0 = base + kPrologue * lane;
 #pragma unroll
-        for (int i = 0; i < kPrologue; ++i) E += k0 + i < a.nb ? __ldg(a.bsum + k0 + i) : 0;
-    }
-    E = __reduce_add_sync(0xffffffffu, E);
+            for (int i = 0; i < kPrologue; ++i) sum += k0 + i < a.nb ? __ldg(a.bsum + k0 + i) : 0;
+        }
+        E = __reduce_add_sync(0xffffffffu, sum);
+        confirmed = true;
+    };
     int t = 0;   // the tile the main loop consumes first
-    // A speculative tile that is not used is left to complete while the walk restarts at tile 1;
-    // stage 0 is waited for before its next use or before the warp exits.
+    // A speculative tile that is not used (the early check) is left to complete while the walk
+    // restarts at tile 1; stage 0 is waited for before its next use or before the warp exits.
     bool spec_pending = false;
     auto drain_spec = [&]() -> bool {
         if (!spec_pending) return true;
@@ -773,21 +840,14 @@ __global__ void __launch_bounds__(32) sparse_decode_kernel(DecodeArgs a, const _
         if (!done && lane == 0) report(a.status, SD_ERR_TIMEOUT);
         return done;
     };
-    if (!(spec && E == e_full)) {
-        if (spec) {
-            spec_pending = true;
-            t = 1;
-        }
-        if (E == 0) {
-            drain_spec();
-            return;
-        }
+    // The split on the row lengths (E entries), its first tile numbered t; false: no entries here.
+    auto start_ragged = [&]() -> bool {
+        if (E == 0) return false;
         w.full = false;
         w.epw = max(a.min_epw, (int)(((long)E + a.total_warps - 1) / a.total_warps));
         const long e0 = (long)blockIdx.x * w.epw;
         if (e0 >= E) {
-            drain_spec();
-            return;
+            return false;
         }
         w.e = (int)e0;
         w.e_end = (int)min((long)E, e0 + w.epw);
@@ -826,8 +886,7 @@ __global__ void __launch_bounds__(32) sparse_decode_kernel(DecodeArgs a, const _
             }
         }
         if (blk < 0) {   // not reached: w.e < E
-            drain_spec();
-            return;
+            return false;
         }
         if (a.rpc == 1) {      // one row per CTA of the row pass
             enter_row(a, w, blk, blk0, blen);
@@ -837,14 +896,27 @@ __global__ void __launch_bounds__(32) sparse_decode_kernel(DecodeArgs a, const _
             const int incl = warp_inclusive_scan(v);
             const uint32_t hit = __ballot_sync(0xffffffffu, blk0 + incl > w.e);
             if (hit == 0u) {   // not reached: the CTA's rows hold entry w.e
-                drain_spec();
-                return;
+                return false;
             }
             const int l = __ffs(hit) - 1;
             enter_row(a, w, r0 + l, blk0 + __shfl_sync(0xffffffffu, incl - v, l), __shfl_sync(0xffffffffu, v, l));
         }
         w.seq = t;
         start_pipeline();
+        return true;
+    };
+    if (!spec || a.weighted) {
+        wait_rows();
+        if (!(spec && E == e_full)) {
+            if (spec) {
+                spec_pending = true;
+                t = 1;
+            }
+            if (!start_ragged()) {
+                drain_spec();
+                return;
+            }
+        }
     }
     // Software pipeline over tiles, so that no load but the gather itself is waited for: while tile
     // t is consumed, tile t + 1 is gathered (its pages were looked up a step earlier), the pages of
@@ -866,11 +938,37 @@ __global__ void __launch_bounds__(32) sparse_decode_kernel(DecodeArgs a, const _
         issue_row_tile(a, ws, kv0, dA, &kmap, &vmap);   // into the stage tile t - 1 used
         dA = dB;
         dB = dC;
-        dC = next_row_tile(a, w);
+        dC = next_row_tile<kOrder>(a, w);
         lookup_pages(a, dA);
         __syncwarp();
         const int4 info = *reinterpret_cast<const int4*>(ws.info[stage]);
         const int flags = (info.x >> 5) & 7;
+        if (!confirmed && (flags & (kFlagLast | kFlagEnd))) {
+            wait_rows();
+            if (E != e_full) {   // rows shorter than k_max: drain tiles t and t + 1, restart from t + 2
+                // Tile u's stage is waited for with parity (u / 2) & 1, which counts one completed phase
+                // per earlier tile of the stage: a tile without rows (an end tile) armed no phase, so
+                // its phase is completed here by a plain arrival.
+                bool drained = true;
+                for (int u = t; u < t + kSparseStages; ++u) {
+                    const int su = u & (kSparseStages - 1);
+                    if ((ws.info[su][0] & 31) > 0)
+                        drained &= mbar_wait(&ws.full[su], (uint32_t)((u >> 1) & 1));
+                    else if (lane == 0)
+                        mbar_arrive(&ws.full[su]);
+                }
+                if (!__all_sync(0xffffffffu, drained)) {
+                    ok = false;
+                    break;
+                }
+                reset_head(st);
+                st.lw = 0.f;
+                t += kSparseStages;
+                if (!start_ragged()) return;
+                --t;   // the loop's increment brings it back to the restarted walk's first tile
+                continue;
+            }
+        }
         if (flags & kFlagEnd) break;
         if (flags & kFlagFirst) {
             load_q_head(ws.q[stage], st);
@@ -888,6 +986,7 @@ __global__ void __launch_bounds__(32) sparse_decode_kernel(DecodeArgs a, const _
         __syncwarp();   // every lane has read the stage before it is refilled
     }
     drain_spec();
+    if (!confirmed) pdl_wait();
     if (!ok) {
         // A copy never completed: record it, wait (bounded) for this warp's copies still in
         // flight, and return; the rows this warp held are left unwritten.
@@ -1047,10 +1146,11 @@ __device__ __forceinline__ TileDesc prefetch_group_tile(const DecodeArgs& a, Gro
             w.cnt = c;
             w.win = w.nwin = -1;
         }
-        if (kUnion) {
-            using MT = typename std::conditional<NT == 1, uint8_t, uint16_t>::type;
-            const MT* gm = reinterpret_cast<const MT*>(a.umask) + (long)grp * a.n_cap +
-                           (long)(w.ri - grp * a.nrp) * kRange;   // the masks of range ri
+        using MT = typename std::conditional<NT == 1, uint8_t, uint16_t>::type;
+        const MT* gm = kUnion ? reinterpret_cast<const MT*>(a.umask) + (long)grp * a.n_cap +
+                                    (long)(w.ri - grp * a.nrp) * kRange   // the masks of range ri
+                              : nullptr;
+        if (kUnion && !a.union_tiles) {
             const int wo = w.off & ~31;
             if (w.win != wo) {   // enter the window: from the prefetch, else loaded now
                 w.wmk = (w.nwin == wo) ? w.nmk : (wo + lane < w.cnt ? (uint32_t)__ldg(gm + wo + lane) : 0u);
@@ -1068,14 +1168,18 @@ __device__ __forceinline__ TileDesc prefetch_group_tile(const DecodeArgs& a, Gro
             uint32_t take = __ballot_sync(0xffffffffu, at >= w.off && at < limit && w.wmk != 0u);
             int consumed = limit - w.off;
             const int need = kTileRows - filled;
+            // one run of selected positions (a window the group selected in full): the i-th selected
+            // position is the run's start + i, no bit search needed
+            const int low = __ffs(take) - 1;
+            const bool run = take != 0u && ((take + (1u << low)) & take) == 0u;
             if (__popc(take) > need) {   // the tile fills up: stop after the need-th selected position
-                const int last = (int)__fns(take, 0, need);
+                const int last = run ? low + need - 1 : (int)__fns(take, 0, need);
                 take &= last == 31 ? 0xffffffffu : ((2u << last) - 1u);
                 consumed = wo + last + 1 - w.off;
             }
             const int cnt = __popc(take);
             const bool mine = lane >= filled && lane < filled + cnt;
-            const int src = mine ? (int)__fns(take, 0, lane - filled + 1) : 0;
+            const int src = mine ? (run ? low + lane - filled : (int)__fns(take, 0, lane - filled + 1)) : 0;
             const uint32_t msrc = __shfl_sync(0xffffffffu, w.wmk, src);
             if (mine) {
                 const int p = (w.ri - grp * a.nrp) * kRange + wo + src;
@@ -1101,14 +1205,20 @@ __device__ __forceinline__ TileDesc prefetch_group_tile(const DecodeArgs& a, Gro
         if (lane >= filled && lane < filled + take) {
             const int off = w.off + lane - filled;
             const int p = (w.ri - grp * a.nrp) * kRange + off;
+            // group walk in whole tiles (the union covers nearly every position): a position no head
+            // selected is not gathered (zero-filled, masked for every head).  The mask and the page
+            // entry are loaded together, before either is examined.
             const int page = __ldg(a.page_table + (long)b * a.max_pages + p / kPageSize);
-            if (page < 0 || page >= a.num_pages) {
+            const uint32_t m = kUnion ? (uint32_t)__ldg(gm + off) : full_mask;
+            if (m == 0u) {
+                d.row_idx = kNoRow;
+            } else if (page < 0 || page >= a.num_pages) {   // (only a selected position's entry is checked)
                 report(a.status, SD_ERR_INDEX_OOB);
                 d.row_idx = kNoRow;
             } else {
                 d.row_idx = ((uint32_t)page * kPageSize + (uint32_t)(p & (kPageSize - 1))) * (uint32_t)a.Hkv + kvh;
             }
-            d.mask = full_mask;
+            d.mask = m;
         }
         filled += take;
         w.off += take;
@@ -1388,9 +1498,17 @@ static cudaError_t occupancy_of(K kernel, int* ctas) {
 cudaError_t decode_occupancy(bool dense, int G, int* ctas_per_sm) {
     if (!dense) {
         const size_t smem = sparse_decode_smem();
-        cudaError_t e = cudaFuncSetAttribute(sparse_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaError_t e = cudaFuncSetAttribute(sparse_decode_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(sparse_decode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, sparse_decode_kernel, 32, smem);
+        int ordered = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&ordered, sparse_decode_kernel<true>, 32, smem);
+        if (e != cudaSuccess) return e;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, sparse_decode_kernel<false>, 32, smem);
+        if (e == cudaSuccess && ordered < *ctas_per_sm) *ctas_per_sm = ordered;
+        return e;
     }
     // (the group walk over selected positions runs with the same shared memory and occupancy)
     int union_ctas = 0;
@@ -1461,20 +1579,30 @@ cudaError_t row_tensor_maps(const DecodeArgs& a, CUtensorMap* kmap, CUtensorMap*
 
 }  // namespace
 
+// The row pass: rows longer than two passes of the CTA's threads keep four passes of loads in flight.
+cudaError_t launch_rows(const DecodeArgs& a, cudaStream_t stream) {
+    const bool deep = (long)a.k_max > 2L * a.tpr * kRowBatch;
+    return deep ? launch_pdl(rows_kernel<4>, dim3(a.nb), dim3(a.tpr * a.rpc), 0, stream, a)
+                : launch_pdl(rows_kernel<1>, dim3(a.nb), dim3(a.tpr * a.rpc), 0, stream, a);
+}
+
 cudaError_t launch_sparse(const DecodeArgs& a, cudaStream_t stream) {
     CUtensorMap kmap, vmap;
     cudaError_t e = row_tensor_maps(a, &kmap, &vmap);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(rows_kernel, dim3(a.nb), dim3(a.tpr * a.rpc), 0, stream, a);
+    e = launch_rows(a, stream);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(sparse_decode_kernel, dim3(a.total_warps), dim3(32), sparse_decode_smem(), stream, a, kmap, vmap);
+    e = a.order_rows
+            ? launch_pdl(sparse_decode_kernel<true>, dim3(a.total_warps), dim3(32), sparse_decode_smem(), stream, a, kmap, vmap)
+            : launch_pdl(sparse_decode_kernel<false>, dim3(a.total_warps), dim3(32), sparse_decode_smem(), stream, a, kmap,
+                         vmap);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 // Sparse decode over GQA groups (rows many heads of a group share): row checks, the groups'
 // selection masks, the group walk over the selected positions, the merge of the segments.
 cudaError_t launch_sparse_union(const DecodeArgs& a, cudaStream_t stream) {
-    cudaError_t e = launch_pdl(rows_kernel, dim3(a.nb), dim3(a.tpr * a.rpc), 0, stream, a);
+    cudaError_t e = launch_rows(a, stream);
     if (e != cudaSuccess) return e;
     e = a.G <= 8 ? launch_pdl(union_masks_kernel<uint8_t>, dim3((unsigned)a.nrt), dim3(256), 0, stream, a)
                  : launch_pdl(union_masks_kernel<uint16_t>, dim3((unsigned)a.nrt), dim3(256), 0, stream, a);

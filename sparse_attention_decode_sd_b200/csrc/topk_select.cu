@@ -16,6 +16,7 @@
 namespace sd {
 
 constexpr int kSelectThreads = 512;
+constexpr int kGatherLoads = 8;   // candidate scores a thread loads together (4096 per CTA and round)
 
 
 // The candidates of row (b, h) as the score pass left them: per page p, the record
@@ -256,26 +257,35 @@ __global__ void __launch_bounds__(kSelectThreads, 2) select_kernel(TopkArgs a) {
         __syncthreads();
         select_masked(RecomputedRow(a, bh, n, qs), take, row, hist, scratch, s_sel);
     } else if (total <= a.cap) {
-        // the usual case: every thread gathers scores for the staged stream indices, four loads in flight
+        // the usual case: every thread gathers scores for the staged stream indices (kGatherLoads loads
+        // in flight) and notes the range of the keys it writes
+        reset_key_range(s_sel);
         __syncthreads();
-        for (int j0 = tid; j0 < total; j0 += 4 * nthr) {
-            uint32_t ix[4];
-            float v[4];
+        uint32_t kmin = 0xffffffffu, kmax = 0u;
+        for (int j0 = tid; j0 < total; j0 += kGatherLoads * nthr) {
+            uint32_t ix[kGatherLoads];
+            float v[kGatherLoads];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < kGatherLoads; ++u) {
                 const int j = j0 + u * nthr;
                 ix[u] = j < total ? lkey[j] : 0xffffffffu;
             }
 #pragma unroll
-            for (int u = 0; u < 4; ++u) v[u] = ix[u] < src.limit ? __ldg(a.cand + ix[u]) : 0.f;
+            for (int u = 0; u < kGatherLoads; ++u) v[u] = ix[u] < src.limit ? __ldg(a.cand + ix[u]) : 0.f;
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < kGatherLoads; ++u) {
                 const int j = j0 + u * nthr;
-                if (j < total) lkey[j] = ix[u] < src.limit ? float_key(v[u]) : 0u;
+                if (j < total) {
+                    const uint32_t key = ix[u] < src.limit ? float_key(v[u]) : 0u;
+                    lkey[j] = key;
+                    kmin = min(kmin, key);
+                    kmax = max(kmax, key);
+                }
             }
         }
+        add_key_range(s_sel, kmin, kmax);
         __syncthreads();
-        select_exact(SharedKeys{lkey, lpos, total}, take, row, hist, scratch, s_sel);
+        select_exact(SharedKeys{lkey, lpos, total}, take, row, hist, scratch, s_sel, true);
     } else {
         select_masked(src, take, row, hist, scratch, s_sel);
     }

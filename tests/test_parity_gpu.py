@@ -122,12 +122,18 @@ def test_decode_repeated_calls_reuse_the_workspace():
 
 
 GROUP_WALK = [
-    # B, Hq, Hkv, lens, k_max, per-head fraction selected: heads of a group that share most rows
-    # make the decode walk groups (one gathered row serves every head that selected it)
-    (2, 16, 4, [20000, 7000], 12000, 0.6),    # two 16384-position ranges, ragged
-    (1, 32, 2, [40000], 30000, 0.7),          # G = 16 (16-bit head masks)
-    (3, 8, 2, [50000, 0, 333], 25000, 0.5),   # an empty request and a short one
-    (2, 8, 4, [17000, 16384], 16384, 1.0),    # G = 2, k = N: every row, range edges
+    # B, Hq, Hkv, lens, k_max, per-head fraction selected: heads of a group that share many rows
+    # (expected duplication G f / (1 - (1 - f)^G) >= 1.4 with f = k_max / capacity) make the decode
+    # walk groups (one gathered row serves every head that selected it).  Where the union is expected
+    # to cover >= 90% of the positions the walk takes whole tiles with head masks, else only the
+    # selected positions.
+    (2, 16, 4, [20000, 7000], 12000, 0.6),    # whole tiles: two 16384-position ranges, ragged
+    (1, 32, 2, [40000], 30000, 0.7),          # whole tiles, G = 16 (16-bit head masks)
+    (3, 8, 2, [50000, 0, 333], 25000, 0.5),   # whole tiles: an empty request and a short one
+    (2, 8, 4, [17000, 16384], 16384, 1.0),    # whole tiles, G = 2, k = N: every row, range edges
+    (2, 16, 2, [30000, 9000], 4500, 0.15),    # selected positions only (coverage 0.73), G = 8
+    (1, 8, 2, [20000], 7000, 0.35),           # selected positions only (coverage 0.82), G = 4
+    (1, 32, 2, [40000], 4000, 0.1),           # selected positions only, G = 16 (16-bit masks)
 ]
 
 

@@ -148,6 +148,47 @@ def test_quest_last_page_update_after_append():
             assert torch.equal(boxes[page], full[page]), (b, j)
 
 
+def test_quest_append_keeps_boxes_current():
+    """sd_quest_append_kv over 20 steps (rows that open new pages and rows that extend them): every box
+    equals the one a full summary of the grown cache writes, bit for bit; K, V and lens as sd_append_kv."""
+    w_cpu = wl.make_workload(3, 8, 2, [40, 47, 48], [16, 16, 16], seed=78, extra_pages=3)
+    k_max = 96
+    w = w_cpu.to(DEV)
+    w2 = w_cpu.to(DEV)
+    shape = sdb.make_shape(w.B, w.Hq, w.Hkv, w.max_pages, k_max, w.num_pages)
+    boxes = sdb.quest_boxes_for(shape, DEV)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    sdb.sd_quest_summarize(shape, w.K, w.page_table, w.lens, boxes, st)
+    g = torch.Generator().manual_seed(4)
+    ks = torch.zeros(w.B, dtype=torch.int32, device=DEV)
+    ks2 = torch.zeros(w.B, dtype=torch.int32, device=DEV)
+    for _ in range(20):
+        kn = torch.randn(w.B, w.Hkv, 128, generator=g).to(torch.bfloat16).to(DEV)
+        vn = torch.randn(w.B, w.Hkv, 128, generator=g).to(torch.bfloat16).to(DEV)
+        sdb.sd_quest_append_kv(shape, w.K, w.V, w.page_table, w.lens, kn, vn, ks, 50, boxes, st)
+        sdb.sd_append_kv(shape, w2.K, w2.V, w2.page_table, w2.lens, kn, vn, ks2, 50, st)
+    full = sdb.quest_boxes_for(shape, DEV)
+    sdb.sd_quest_summarize(shape, w.K, w.page_table, w.lens, full, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert torch.equal(w.K, w2.K) and torch.equal(w.V, w2.V) and torch.equal(w.lens, w2.lens) and torch.equal(ks, ks2)
+    assert [int(x) for x in w.lens] == [60, 67, 68]
+    for b in range(w.B):
+        n = int(w.lens[b])
+        for j in range((n + P - 1) // P):
+            page = int(w.page_table[b, j])
+            assert torch.equal(boxes[page], full[page]), (b, j)
+
+
+def test_quest_append_rejects_missing_boxes():
+    w = wl.make_workload(1, 8, 2, [40], [16], seed=79, extra_pages=1).to(DEV)
+    shape = sdb.make_shape(w.B, w.Hq, w.Hkv, w.max_pages, 64, w.num_pages)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    kn = torch.zeros(w.B, w.Hkv, 128, dtype=torch.bfloat16, device=DEV)
+    assert sdb.sd_quest_append_kv(shape, w.K, w.V, w.page_table, w.lens, kn, kn, None, 50, None, st,
+                                  check=False) == sdb.SD_ERR_INVALID_ARG
+
+
 def test_quest_long128k_sampled():
     """The benchmark's workload (4 x 64/8 heads, N = 131072, k = 2621): Quest pages on sampled groups."""
     w = wl.named("long128k", device=DEV)
