@@ -808,30 +808,19 @@ __global__ void __launch_bounds__(32) sparse_decode_kernel(DecodeArgs a, const _
         enter_row(a, w, row_of_slot<kOrder>(a, w, slot), slot * a.k_max, a.k_max);
         start_pipeline();
     }
-    // The row pass's results -- row checks, lengths, zeroed arrival counters, drawn-row weights -- are
-    // needed before this warp's first global write (a segment's partial or a row's output) and before
-    // any read of them.  A warp on the full-row split waits only then (at its first segment end),
-    // with its first tiles already consumed; the entry count E = R * k_max confirms its split, else
-    // the tiles in flight are drained and the walk restarts on the row lengths.  Weighted mode reads
-    // the drawn-row weights when a row opens, so it waits before the loop.
+    pdl_wait();   // rows_kernel: row lengths, checks, zeroed arrival counters
+    // E = all entries: the length sums of the rows_kernel CTAs, each lane summing kPrologue
+    // consecutive ones per round
     int E = 0;
-    bool confirmed = false;
-    auto wait_rows = [&]() {
-        pdl_wait();
-        // E = all entries: the length sums of the rows_kernel CTAs, each lane summing kPrologue
-        // consecutive ones per round
-        int sum = 0;
-        for (int base = 0; base < a.nb; base += 32 * kPrologue) {
-            const int k0 = base + kPrologue * lane;
+    for (int base = 0; base < a.nb; base += 32 * kPrologue) {
+        const int k0 = base + kPrologue * lane;
 #pragma unroll
-            for (int i = 0; i < kPrologue; ++i) sum += k0 + i < a.nb ? __ldg(a.bsum + k0 + i) : 0;
-        }
-        E = __reduce_add_sync(0xffffffffu, sum);
-        confirmed = true;
-    };
+        for (int i = 0; i < kPrologue; ++i) E += k0 + i < a.nb ? __ldg(a.bsum + k0 + i) : 0;
+    }
+    E = __reduce_add_sync(0xffffffffu, E);
     int t = 0;   // the tile the main loop consumes first
-    // A speculative tile that is not used (the early check) is left to complete while the walk
-    // restarts at tile 1; stage 0 is waited for before its next use or before the warp exits.
+    // A speculative tile that is not used is left to complete while the walk restarts at tile 1;
+    // stage 0 is waited for before its next use or before the warp exits.
     bool spec_pending = false;
     auto drain_spec = [&]() -> bool {
         if (!spec_pending) return true;
@@ -840,14 +829,21 @@ __global__ void __launch_bounds__(32) sparse_decode_kernel(DecodeArgs a, const _
         if (!done && lane == 0) report(a.status, SD_ERR_TIMEOUT);
         return done;
     };
-    // The split on the row lengths (E entries), its first tile numbered t; false: no entries here.
-    auto start_ragged = [&]() -> bool {
-        if (E == 0) return false;
+    if (!(spec && E == e_full)) {
+        if (spec) {
+            spec_pending = true;
+            t = 1;
+        }
+        if (E == 0) {
+            drain_spec();
+            return;
+        }
         w.full = false;
         w.epw = max(a.min_epw, (int)(((long)E + a.total_warps - 1) / a.total_warps));
         const long e0 = (long)blockIdx.x * w.epw;
         if (e0 >= E) {
-            return false;
+            drain_spec();
+            return;
         }
         w.e = (int)e0;
         w.e_end = (int)min((long)E, e0 + w.epw);
@@ -886,7 +882,8 @@ __global__ void __launch_bounds__(32) sparse_decode_kernel(DecodeArgs a, const _
             }
         }
         if (blk < 0) {   // not reached: w.e < E
-            return false;
+            drain_spec();
+            return;
         }
         if (a.rpc == 1) {      // one row per CTA of the row pass
             enter_row(a, w, blk, blk0, blen);
@@ -896,27 +893,14 @@ __global__ void __launch_bounds__(32) sparse_decode_kernel(DecodeArgs a, const _
             const int incl = warp_inclusive_scan(v);
             const uint32_t hit = __ballot_sync(0xffffffffu, blk0 + incl > w.e);
             if (hit == 0u) {   // not reached: the CTA's rows hold entry w.e
-                return false;
+                drain_spec();
+                return;
             }
             const int l = __ffs(hit) - 1;
             enter_row(a, w, r0 + l, blk0 + __shfl_sync(0xffffffffu, incl - v, l), __shfl_sync(0xffffffffu, v, l));
         }
         w.seq = t;
         start_pipeline();
-        return true;
-    };
-    if (!spec || a.weighted) {
-        wait_rows();
-        if (!(spec && E == e_full)) {
-            if (spec) {
-                spec_pending = true;
-                t = 1;
-            }
-            if (!start_ragged()) {
-                drain_spec();
-                return;
-            }
-        }
     }
     // Software pipeline over tiles, so that no load but the gather itself is waited for: while tile
     // t is consumed, tile t + 1 is gathered (its pages were looked up a step earlier), the pages of
@@ -943,32 +927,6 @@ __global__ void __launch_bounds__(32) sparse_decode_kernel(DecodeArgs a, const _
         __syncwarp();
         const int4 info = *reinterpret_cast<const int4*>(ws.info[stage]);
         const int flags = (info.x >> 5) & 7;
-        if (!confirmed && (flags & (kFlagLast | kFlagEnd))) {
-            wait_rows();
-            if (E != e_full) {   // rows shorter than k_max: drain tiles t and t + 1, restart from t + 2
-                // Tile u's stage is waited for with parity (u / 2) & 1, which counts one completed phase
-                // per earlier tile of the stage: a tile without rows (an end tile) armed no phase, so
-                // its phase is completed here by a plain arrival.
-                bool drained = true;
-                for (int u = t; u < t + kSparseStages; ++u) {
-                    const int su = u & (kSparseStages - 1);
-                    if ((ws.info[su][0] & 31) > 0)
-                        drained &= mbar_wait(&ws.full[su], (uint32_t)((u >> 1) & 1));
-                    else if (lane == 0)
-                        mbar_arrive(&ws.full[su]);
-                }
-                if (!__all_sync(0xffffffffu, drained)) {
-                    ok = false;
-                    break;
-                }
-                reset_head(st);
-                st.lw = 0.f;
-                t += kSparseStages;
-                if (!start_ragged()) return;
-                --t;   // the loop's increment brings it back to the restarted walk's first tile
-                continue;
-            }
-        }
         if (flags & kFlagEnd) break;
         if (flags & kFlagFirst) {
             load_q_head(ws.q[stage], st);
@@ -986,7 +944,6 @@ __global__ void __launch_bounds__(32) sparse_decode_kernel(DecodeArgs a, const _
         __syncwarp();   // every lane has read the stage before it is refilled
     }
     drain_spec();
-    if (!confirmed) pdl_wait();
     if (!ok) {
         // A copy never completed: record it, wait (bounded) for this warp's copies still in
         // flight, and return; the rows this warp held are left unwritten.

@@ -16,7 +16,6 @@
 namespace sd {
 
 constexpr int kSelectThreads = 512;
-constexpr int kGatherLoads = 8;   // candidate scores a thread loads together (4096 per CTA and round)
 
 
 // The candidates of row (b, h) as the score pass left them: per page p, the record
@@ -257,35 +256,26 @@ __global__ void __launch_bounds__(kSelectThreads, 2) select_kernel(TopkArgs a) {
         __syncthreads();
         select_masked(RecomputedRow(a, bh, n, qs), take, row, hist, scratch, s_sel);
     } else if (total <= a.cap) {
-        // the usual case: every thread gathers scores for the staged stream indices (kGatherLoads loads
-        // in flight) and notes the range of the keys it writes
-        reset_key_range(s_sel);
+        // the usual case: every thread gathers scores for the staged stream indices, four loads in flight
         __syncthreads();
-        uint32_t kmin = 0xffffffffu, kmax = 0u;
-        for (int j0 = tid; j0 < total; j0 += kGatherLoads * nthr) {
-            uint32_t ix[kGatherLoads];
-            float v[kGatherLoads];
+        for (int j0 = tid; j0 < total; j0 += 4 * nthr) {
+            uint32_t ix[4];
+            float v[4];
 #pragma unroll
-            for (int u = 0; u < kGatherLoads; ++u) {
+            for (int u = 0; u < 4; ++u) {
                 const int j = j0 + u * nthr;
                 ix[u] = j < total ? lkey[j] : 0xffffffffu;
             }
 #pragma unroll
-            for (int u = 0; u < kGatherLoads; ++u) v[u] = ix[u] < src.limit ? __ldg(a.cand + ix[u]) : 0.f;
+            for (int u = 0; u < 4; ++u) v[u] = ix[u] < src.limit ? __ldg(a.cand + ix[u]) : 0.f;
 #pragma unroll
-            for (int u = 0; u < kGatherLoads; ++u) {
+            for (int u = 0; u < 4; ++u) {
                 const int j = j0 + u * nthr;
-                if (j < total) {
-                    const uint32_t key = ix[u] < src.limit ? float_key(v[u]) : 0u;
-                    lkey[j] = key;
-                    kmin = min(kmin, key);
-                    kmax = max(kmax, key);
-                }
+                if (j < total) lkey[j] = ix[u] < src.limit ? float_key(v[u]) : 0u;
             }
         }
-        add_key_range(s_sel, kmin, kmax);
         __syncthreads();
-        select_exact(SharedKeys{lkey, lpos, total}, take, row, hist, scratch, s_sel, true);
+        select_exact(SharedKeys{lkey, lpos, total}, take, row, hist, scratch, s_sel);
     } else {
         select_masked(src, take, row, hist, scratch, s_sel);
     }
