@@ -75,13 +75,16 @@ struct __align__(128) DecodeSmem {
 
 size_t decode_smem() { return sizeof(DecodeSmem); }
 
-// A tile fetched one iteration ahead: row descriptors live in lanes 0..15.
+// A tile fetched one iteration ahead: row descriptors live in lanes 0..15.  The page entry and the
+// head mask are loads that the prefetch only issues; they are first examined when the tile is issued,
+// an iteration later, so that the warp computes the tile in between without waiting for them.
 struct TileDesc {
     int rows, flags;
     int owner;          // dense: group b * Hkv + kvh; sparse: row b * Hq + h
     int seg_j, nseg;    // segment slot of this warp in the owner, and the owner's segment count (sparse)
-    uint32_t row_idx;   // this lane's cache row (lanes < rows); kNoRow: none (the row is skipped)
-    uint32_t mask;      // heads (columns) that attend to it
+    int page;           // this lane's page-table entry (lanes < rows)
+    uint32_t sub;       // this lane's row within the page block: slot * Hkv + kvh
+    uint32_t mask;      // heads (columns) that attend to it (0: none, the row is not gathered)
 };
 
 __device__ __forceinline__ TileDesc empty_tile() {
@@ -89,7 +92,8 @@ __device__ __forceinline__ TileDesc empty_tile() {
     d.rows = 0;
     d.flags = 0;
     d.owner = d.seg_j = d.nseg = 0;
-    d.row_idx = 0;
+    d.page = 0;
+    d.sub = 0;
     d.mask = 0;
     return d;
 }
@@ -100,7 +104,13 @@ __device__ __forceinline__ TileDesc empty_tile() {
 // iteration earlier, so that load stays in flight while the warp computes the previous tile.
 __device__ __forceinline__ void issue_tile(const DecodeArgs& a, DecodeSmem& ws, int stage, const TileDesc& d) {
     const int lane = threadIdx.x & 31;
-    if (lane < kTileRows) ws.meta_mask[stage][lane] = (lane < d.rows && d.row_idx != kNoRow) ? d.mask : 0u;
+    // this lane's cache row: a selected row whose page entry is outside the cache is reported and skipped
+    const bool sel = lane < d.rows && d.mask != 0u;
+    const bool bad = sel && (d.page < 0 || d.page >= a.num_pages);
+    if (bad) report(a.status, SD_ERR_INDEX_OOB);
+    const uint32_t row_idx =
+        (sel && !bad) ? (uint32_t)d.page * (uint32_t)(kPageSize * a.Hkv) + d.sub : kNoRow;
+    if (lane < kTileRows) ws.meta_mask[stage][lane] = row_idx != kNoRow ? d.mask : 0u;
     if (lane == 0) {
         ws.info[stage][0] = d.rows;
         ws.info[stage][1] = d.flags;
@@ -117,7 +127,7 @@ __device__ __forceinline__ void issue_tile(const DecodeArgs& a, DecodeSmem& ws, 
 #pragma unroll
         for (int i = 0; i < kTileRows / 2; ++i) {
             const int r = (lane >> 4) + 2 * i;
-            const uint32_t ri = __shfl_sync(0xffffffffu, d.row_idx, r);
+            const uint32_t ri = __shfl_sync(0xffffffffu, row_idx, r);
             const bool ok = r < d.rows && ri != kNoRow;
             const size_t off = ok ? (((size_t)ri << 8) + (ch << 4)) : 0;
             const uint32_t doff = (uint32_t)(r * kRowPitch + (ch << 4));
@@ -1140,13 +1150,8 @@ __device__ __forceinline__ TileDesc prefetch_group_tile(const DecodeArgs& a, Gro
             const uint32_t msrc = __shfl_sync(0xffffffffu, w.wmk, src);
             if (mine) {
                 const int p = (w.ri - grp * a.nrp) * kRange + wo + src;
-                const int page = __ldg(a.page_table + (long)b * a.max_pages + p / kPageSize);
-                if (page < 0 || page >= a.num_pages) {
-                    report(a.status, SD_ERR_INDEX_OOB);
-                    d.row_idx = kNoRow;
-                } else {
-                    d.row_idx = ((uint32_t)page * kPageSize + (uint32_t)(p & (kPageSize - 1))) * (uint32_t)a.Hkv + kvh;
-                }
+                d.page = __ldg(a.page_table + (long)b * a.max_pages + p / kPageSize);
+                d.sub = (uint32_t)(p & (kPageSize - 1)) * (uint32_t)a.Hkv + kvh;
                 d.mask = msrc;
             }
             filled += cnt;
@@ -1163,19 +1168,10 @@ __device__ __forceinline__ TileDesc prefetch_group_tile(const DecodeArgs& a, Gro
             const int off = w.off + lane - filled;
             const int p = (w.ri - grp * a.nrp) * kRange + off;
             // group walk in whole tiles (the union covers nearly every position): a position no head
-            // selected is not gathered (zero-filled, masked for every head).  The mask and the page
-            // entry are loaded together, before either is examined.
-            const int page = __ldg(a.page_table + (long)b * a.max_pages + p / kPageSize);
-            const uint32_t m = kUnion ? (uint32_t)__ldg(gm + off) : full_mask;
-            if (m == 0u) {
-                d.row_idx = kNoRow;
-            } else if (page < 0 || page >= a.num_pages) {   // (only a selected position's entry is checked)
-                report(a.status, SD_ERR_INDEX_OOB);
-                d.row_idx = kNoRow;
-            } else {
-                d.row_idx = ((uint32_t)page * kPageSize + (uint32_t)(p & (kPageSize - 1))) * (uint32_t)a.Hkv + kvh;
-            }
-            d.mask = m;
+            // selected (mask 0) is not gathered -- zero-filled and masked for every head
+            d.page = __ldg(a.page_table + (long)b * a.max_pages + p / kPageSize);
+            d.sub = (uint32_t)(p & (kPageSize - 1)) * (uint32_t)a.Hkv + kvh;
+            d.mask = kUnion ? (uint32_t)__ldg(gm + off) : full_mask;
         }
         filled += take;
         w.off += take;
