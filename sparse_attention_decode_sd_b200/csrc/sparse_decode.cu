@@ -75,16 +75,19 @@ struct __align__(128) DecodeSmem {
 
 size_t decode_smem() { return sizeof(DecodeSmem); }
 
-// A tile fetched one iteration ahead: row descriptors live in lanes 0..15.  The page entry and the
-// head mask are loads that the prefetch only issues; they are first examined when the tile is issued,
-// an iteration later, so that the warp computes the tile in between without waiting for them.
+// A tile fetched one iteration ahead: row descriptors live in lanes 0..15.  Dense walk: the cache row
+// is worked out at the prefetch (the page-table entry comes from L2).  Group walk: the page entry and
+// the head mask (which comes from DRAM) are loads that the prefetch only issues; they are first
+// examined when the tile is issued, an iteration later, so that the warp computes the tile in between
+// without waiting for them.
 struct TileDesc {
     int rows, flags;
     int owner;          // dense: group b * Hkv + kvh; sparse: row b * Hq + h
     int seg_j, nseg;    // segment slot of this warp in the owner, and the owner's segment count (sparse)
-    int page;           // this lane's page-table entry (lanes < rows)
-    uint32_t sub;       // this lane's row within the page block: slot * Hkv + kvh
-    uint32_t mask;      // heads (columns) that attend to it (0: none, the row is not gathered)
+    uint32_t row_idx;   // dense walk: this lane's cache row (lanes < rows); kNoRow: none (skipped)
+    int page;           // group walk: this lane's page-table entry (lanes < rows)
+    uint32_t sub;       // group walk: this lane's row within the page block, slot * Hkv + kvh
+    uint32_t mask;      // heads (columns) that attend to it (group walk, 0: none, the row is not gathered)
 };
 
 __device__ __forceinline__ TileDesc empty_tile() {
@@ -92,6 +95,7 @@ __device__ __forceinline__ TileDesc empty_tile() {
     d.rows = 0;
     d.flags = 0;
     d.owner = d.seg_j = d.nseg = 0;
+    d.row_idx = 0;
     d.page = 0;
     d.sub = 0;
     d.mask = 0;
@@ -102,15 +106,17 @@ __device__ __forceinline__ TileDesc empty_tile() {
 // copying chunk l % 16 of rows l / 16, l / 16 + 2, ...; missing rows are zero-filled.  One
 // cp.async group per tile.  This is the first use of the row indices loaded by the prefetch one
 // iteration earlier, so that load stays in flight while the warp computes the previous tile.
+template <bool kUnion>
 __device__ __forceinline__ void issue_tile(const DecodeArgs& a, DecodeSmem& ws, int stage, const TileDesc& d) {
     const int lane = threadIdx.x & 31;
-    // this lane's cache row: a selected row whose page entry is outside the cache is reported and skipped
-    const bool sel = lane < d.rows && d.mask != 0u;
-    const bool bad = sel && (d.page < 0 || d.page >= a.num_pages);
-    if (bad) report(a.status, SD_ERR_INDEX_OOB);
-    const uint32_t row_idx =
-        (sel && !bad) ? (uint32_t)d.page * (uint32_t)(kPageSize * a.Hkv) + d.sub : kNoRow;
-    if (lane < kTileRows) ws.meta_mask[stage][lane] = row_idx != kNoRow ? d.mask : 0u;
+    uint32_t row_idx = d.row_idx;
+    if (kUnion) {   // a selected row whose page entry is outside the cache is reported and skipped
+        const bool sel = lane < d.rows && d.mask != 0u;
+        const bool bad = sel && (d.page < 0 || d.page >= a.num_pages);
+        if (bad) report(a.status, SD_ERR_INDEX_OOB);
+        row_idx = (sel && !bad) ? (uint32_t)d.page * (uint32_t)(kPageSize * a.Hkv) + d.sub : kNoRow;
+    }
+    if (lane < kTileRows) ws.meta_mask[stage][lane] = (lane < d.rows && row_idx != kNoRow) ? d.mask : 0u;
     if (lane == 0) {
         ws.info[stage][0] = d.rows;
         ws.info[stage][1] = d.flags;
@@ -1167,11 +1173,23 @@ __device__ __forceinline__ TileDesc prefetch_group_tile(const DecodeArgs& a, Gro
         if (lane >= filled && lane < filled + take) {
             const int off = w.off + lane - filled;
             const int p = (w.ri - grp * a.nrp) * kRange + off;
-            // group walk in whole tiles (the union covers nearly every position): a position no head
-            // selected (mask 0) is not gathered -- zero-filled and masked for every head
-            d.page = __ldg(a.page_table + (long)b * a.max_pages + p / kPageSize);
-            d.sub = (uint32_t)(p & (kPageSize - 1)) * (uint32_t)a.Hkv + kvh;
-            d.mask = kUnion ? (uint32_t)__ldg(gm + off) : full_mask;
+            if (kUnion) {
+                // group walk in whole tiles (the union covers nearly every position): a position no head
+                // selected (mask 0) is not gathered -- zero-filled and masked for every head
+                d.page = __ldg(a.page_table + (long)b * a.max_pages + p / kPageSize);
+                d.sub = (uint32_t)(p & (kPageSize - 1)) * (uint32_t)a.Hkv + kvh;
+                d.mask = (uint32_t)__ldg(gm + off);
+            } else {
+                const int page = __ldg(a.page_table + (long)b * a.max_pages + p / kPageSize);
+                if (page < 0 || page >= a.num_pages) {
+                    report(a.status, SD_ERR_INDEX_OOB);
+                    d.row_idx = kNoRow;
+                } else {
+                    d.row_idx =
+                        ((uint32_t)page * kPageSize + (uint32_t)(p & (kPageSize - 1))) * (uint32_t)a.Hkv + kvh;
+                }
+                d.mask = full_mask;
+            }
         }
         filled += take;
         w.off += take;
@@ -1313,13 +1331,13 @@ __global__ void __launch_bounds__(32) dense_decode_kernel(DecodeArgs a) {
     TileDesc next = prefetch_group_tile<NT, kUnion>(a, w);
 #pragma unroll
     for (int s = 0; s < kStages - 1; ++s) {
-        issue_tile(a, ws, s, next);
+        issue_tile<kUnion>(a, ws, s, next);
         next = prefetch_group_tile<NT, kUnion>(a, w);
     }
     for (int t = 0;; ++t) {
         const int stage = t % kStages;
         // the stage of tile t-1 is free: issue tile t+kStages-1 before waiting for tile t
-        issue_tile(a, ws, (t + kStages - 1) % kStages, next);
+        issue_tile<kUnion>(a, ws, (t + kStages - 1) % kStages, next);
         next = prefetch_group_tile<NT, kUnion>(a, w);
         cp_async_wait<kStages - 1>();
         __syncwarp();
