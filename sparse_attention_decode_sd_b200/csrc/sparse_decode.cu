@@ -1014,6 +1014,49 @@ __device__ __forceinline__ int first_at_least(const int32_t* row, int len, int t
     return ge ? lo + __ffs(ge) - 1 : hi;
 }
 
+// The group walk's check of idx: every rule a row must follow is one on adjacent entries (positions
+// ascending, below N_b, no position after the first negative entry), so the rows are cut into chunks of
+// kValidateEntries consecutive entries, one thread each, over the whole grid (no per-row reduction:
+// the group walk needs no row lengths).  A chunk whose start is 16-byte aligned is loaded as vectors.
+constexpr int kValidateEntries = 16;
+__global__ void __launch_bounds__(256) validate_kernel(DecodeArgs a) {
+    pdl_enter();
+    const long per_row = (a.k_max + kValidateEntries - 1) / kValidateEntries;
+    const long t = (long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long r = t / per_row;
+    if (r >= (long)a.B * a.Hq) return;
+    const int j0 = (int)(t - r * per_row) * kValidateEntries;
+    const int32_t* row = a.idx + r * a.k_max;
+    const int n = checked_len(a.lens, (int)(r / a.Hq), a.n_cap, a.status);
+    int v[kValidateEntries];
+    const int cnt = min(kValidateEntries, a.k_max - j0);
+    if (cnt == kValidateEntries && (reinterpret_cast<uintptr_t>(row + j0) & 15u) == 0) {
+#pragma unroll
+        for (int i = 0; i < kValidateEntries / 4; ++i) {
+            const int4 q = __ldg(reinterpret_cast<const int4*>(row + j0) + i);
+            v[4 * i] = q.x;
+            v[4 * i + 1] = q.y;
+            v[4 * i + 2] = q.z;
+            v[4 * i + 3] = q.w;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < kValidateEntries; ++i) v[i] = i < cnt ? __ldg(row + j0 + i) : -1;
+    }
+    int p = j0 > 0 ? __ldg(row + j0 - 1) : -1;
+    bool oob = false, order = false;
+#pragma unroll
+    for (int i = 0; i < kValidateEntries; ++i) {
+        if (i < cnt && v[i] >= 0) {
+            oob |= v[i] >= n;
+            order |= (j0 + i > 0) && (p < 0 || p >= v[i]);
+        }
+        p = v[i];
+    }
+    if (oob) report(a.status, SD_ERR_INDEX_OOB);
+    else if (order) report(a.status, SD_ERR_ORDER);
+}
+
 // One CTA per (group, kRange-position range): the heads of the group that selected each position,
 // as bits of a per-position mask (MT: 8 bits for G <= 8, 16 for G <= 16) in the workspace, and the
 // range's position count (the unit the group walk is split in).  Each warp finds a head's entries
@@ -1573,7 +1616,8 @@ cudaError_t launch_sparse(const DecodeArgs& a, cudaStream_t stream) {
 // Sparse decode over GQA groups (rows many heads of a group share): row checks, the groups'
 // selection masks, the group walk over the selected positions, the merge of the segments.
 cudaError_t launch_sparse_union(const DecodeArgs& a, cudaStream_t stream) {
-    cudaError_t e = launch_rows(a, stream);
+    const long chunks = (long)a.B * a.Hq * ((a.k_max + kValidateEntries - 1) / kValidateEntries);
+    cudaError_t e = launch_pdl(validate_kernel, dim3((unsigned)((chunks + 255) / 256)), dim3(256), 0, stream, a);
     if (e != cudaSuccess) return e;
     e = a.G <= 8 ? launch_pdl(union_masks_kernel<uint8_t>, dim3((unsigned)a.nrt), dim3(256), 0, stream, a)
                  : launch_pdl(union_masks_kernel<uint16_t>, dim3((unsigned)a.nrt), dim3(256), 0, stream, a);

@@ -162,6 +162,27 @@ def test_group_walk_arbitrary_rows(B, Hq, Hkv, lens, k_max, frac):
     assert (out[:, 1] == 0).all()
 
 
+@pytest.mark.parametrize("defect,code", [("swap", sdb.SD_ERR_ORDER), ("past_end", sdb.SD_ERR_INDEX_OOB),
+                                         ("after_padding", sdb.SD_ERR_ORDER)])
+def test_group_walk_reports_bad_rows(defect, code):
+    """Rows checked on the group walk's path (k close to N, where it is taken): a swapped pair, a
+    position at N_b and a position after the padding are each reported."""
+    B, Hq, Hkv, n = 2, 8, 4, 16384
+    w_cpu = wl.make_workload(B, Hq, Hkv, n, 1, seed=5, k_max=n)
+    idx = torch.arange(n, dtype=torch.int32).repeat(B, Hq, 1)
+    if defect == "swap":
+        idx[1, 5, 7000], idx[1, 5, 7001] = 7001, 7000
+    elif defect == "past_end":
+        idx[0, 2, n - 1] = n
+    else:
+        idx[1, 6, 9000:] = -1
+        idx[1, 6, 12000] = 12000
+    w = w_cpu.to(DEV)
+    r = gh.Runner(w)
+    r.sparse(idx.to(DEV))
+    assert r.device_status() == code
+
+
 @pytest.mark.parametrize("n,k", [(3000, 100), (40000, 100), (40000, 39999)])
 def test_exact_ties_go_to_lower_positions(n, k):
     """Identical K rows: every score ties, so the selection is exactly positions 0..k-1.  With N
