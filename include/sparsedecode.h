@@ -143,11 +143,16 @@ SD_API sd_status sd_topk_index_static(const sd_shape* shape, const void* q, cons
  * context sparsity"; SDPA of the xllm survey sec. 1.1 restricted to the selected set).
  *   out[b,h] = sum_{i in S} w_i V[b, h/G, i],  w = softmax over S of (q[b,h] . K[b,h/G,i]) / sqrt(d),
  *   S = the entries of idx[b][h] before its first negative one.  An empty S gives out = 0.
- *   Each query head gathers its own rows; the heads of a GQA group are processed side by side, so a
- *   row that several of them selected is read from HBM about once and from L2 after that.
- *   The call launches two kernels; the second starts gathering before the first (the row checks)
- *   ends, so idx, q, K, V and the page table must be complete when the call is enqueued (stream
- *   order), as for every call of the library.
+ *   Two walks, chosen from the shape alone, give the same result up to rounding order:
+ *   - per query head (the usual case): each head gathers its own rows; the heads of a GQA group are
+ *     processed side by side, so a row that several of them selected is read from HBM about once and
+ *     from L2 after that.  Two kernels; the second starts gathering before the first (the row
+ *     checks) ends, so idx, q, K, V and the page table must be complete when the call is enqueued
+ *     (stream order), as for every call of the library.
+ *   - per GQA group, when the heads of a group are expected to share many rows (expected duplication
+ *     G f / (1 - (1 - f)^G) >= 1.4, f = k_max / (max_pages_per_req * 16)): each row of the group's
+ *     union is gathered once for every head that selected it.  Four kernels (row checks, the group's
+ *     head masks, the walk, the merge).
  *   num_pages * 16 * Hkv must be below 2^31 (cache rows are TMA coordinates), else
  *   SD_ERR_UNSUPPORTED.
  *   Device checks: entries must be < N_b and map to a page-table entry in range (SD_ERR_INDEX_OOB),
