@@ -22,6 +22,7 @@ import datetime
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -58,10 +59,14 @@ def peaks():
 
 
 def source_hash(*names):
+    """Hash of the kernels' code: the sources with comments and blank lines removed, so that a capture
+    stays keyed to its code when only comments change."""
     h = hashlib.sha256()
     for n in names:
-        with open(os.path.join(ROOT, "sparse_attention_decode_sd_b200", "csrc", n), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "sparse_attention_decode_sd_b200", "csrc", n), encoding="utf-8") as f:
+            text = re.sub(r"/\*.*?\*/", "", f.read(), flags=re.S)
+        lines = (re.sub(r"//.*", "", line).rstrip() for line in text.splitlines())
+        h.update("\n".join(line for line in lines if line).encode())
     return h.hexdigest()[:16]
 
 

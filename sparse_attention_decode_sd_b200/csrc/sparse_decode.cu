@@ -34,10 +34,12 @@
 //                         by one warp is written out directly.
 //
 // Sparse decode over GQA groups (chosen by the host when the heads of a group are expected to
-// share many rows), four kernels: rows_kernel as above; union_masks_kernel sets, per (group,
-// 16384-position range), a byte (two for G > 8) per position whose bits are the heads that selected
-// it; dense_decode_kernel<., true> walks only the masked positions of every group, one gathered tile
-// serving every head that selected its rows; merge_kernel combines the partials.
+// share many rows), four kernels: validate_kernel checks idx in chunks of 16 entries over the whole
+// grid (every rule is on adjacent entries, and no row lengths are needed); union_masks_kernel sets,
+// per (group, 16384-position range), a byte (two for G > 8) per position whose bits are the heads
+// that selected it; dense_decode_kernel<., true> walks the masked positions of every group -- only
+// those, or whole tiles with their masks where the union covers nearly every position -- one
+// gathered tile serving every head that selected its rows; merge_kernel combines the partials.
 //
 // Dense decode (the comparator), three kernels: ranges_kernel counts the positions of each
 // kRange-position range of every (request, KV head) group; dense_decode_kernel walks all rows of every
@@ -1613,7 +1615,7 @@ cudaError_t launch_sparse(const DecodeArgs& a, cudaStream_t stream) {
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-// Sparse decode over GQA groups (rows many heads of a group share): row checks, the groups'
+// Sparse decode over GQA groups (rows many heads of a group share): the checks of idx, the groups'
 // selection masks, the group walk over the selected positions, the merge of the segments.
 cudaError_t launch_sparse_union(const DecodeArgs& a, cudaStream_t stream) {
     const long chunks = (long)a.B * a.Hq * ((a.k_max + kValidateEntries - 1) / kValidateEntries);
