@@ -88,6 +88,25 @@ def test_workspace_sizes(lib):
     assert sparse % 256 == 0 and dense % 256 == 0 and topk % 256 == 0
 
 
+def test_workspace_size_of_the_group_walk(lib):
+    """A shape whose heads are expected to share most rows (k = N, G = 4) takes the group walk: its
+    workspace holds the per-head walk's part (which a stochastic selection, decoded per head, uses),
+    the dense decode's partials and range counts, and one head-mask byte per position of each group."""
+    B, Hq, Hkv, max_pages, k_max = 4, 32, 8, 1024, 16384
+    s = _shape(B=B, Hq=Hq, Hkv=Hkv, max_pages=max_pages, k_max=k_max, num_pages=B * max_pages)
+    got = sdb.sd_workspace_size(s, sdb.SD_OP_SPARSE)
+    rows = B * Hq
+    per_head = rows * 64 * (128 * 4 + 8) + rows * 4 * 3 + rows * 4   # partials, lengths/counters/weights, sums
+    slots = rows * (1280 + 1)
+    dense = slots * (128 * 4 + 8) + B * Hkv * 1 * 4                    # one 16384-position range per group
+    masks = B * Hkv * max_pages * 16
+    need = per_head + dense + masks
+    assert need <= got <= need + 10 * 256
+    # the same shape at 50x sparsity keeps the per-head walk's workspace alone
+    s50 = _shape(B=B, Hq=Hq, Hkv=Hkv, max_pages=max_pages, k_max=328, num_pages=B * max_pages)
+    assert sdb.sd_workspace_size(s50, sdb.SD_OP_SPARSE) < per_head
+
+
 def test_sparse_workspace_rejects_entry_count_overflow(lib):
     # B * Hq * k_max entries are counted in int32
     n = ctypes.c_size_t(0)
@@ -132,6 +151,17 @@ def test_null_and_misaligned_pointers_rejected_before_launch(lib):
     assert lib.sd_dense_decode(s, fake, fake, fake, fake, fake, fake, N, ws, fake, N) == sdb.SD_ERR_INVALID_ARG
     assert lib.sd_append_kv(s, fake, fake, fake, fake, fake, fake, N, 0, fake, N) == sdb.SD_ERR_INVALID_ARG
     assert lib.sd_append_kv(s, fake, fake, fake, fake, N, fake, N, 50, fake, N) == sdb.SD_ERR_INVALID_ARG
+    # the append that keeps Quest boxes: boxes required and 16-byte aligned, then the append's own checks
+    assert lib.sd_quest_append_kv(s, fake, fake, fake, fake, fake, fake, N, 50, N, fake, N) == sdb.SD_ERR_INVALID_ARG
+    assert lib.sd_quest_append_kv(s, fake, fake, fake, fake, fake, fake, N, 50, odd, fake, N) == sdb.SD_ERR_INVALID_ARG
+    assert lib.sd_quest_append_kv(s, fake, fake, fake, fake, N, fake, N, 50, fake, fake, N) == sdb.SD_ERR_INVALID_ARG
+    # stochastic selection: k_samp required, then the exact indexer's checks (idx null)
+    assert lib.sd_stochastic_index(s, fake, fake, fake, fake, fake, N, 1, 0, fake, fake, ws, fake, N) == \
+        sdb.SD_ERR_INVALID_ARG
+    assert lib.sd_stochastic_index(s, fake, fake, fake, fake, fake, fake, 1, 0, N, fake, ws, fake, N) == \
+        sdb.SD_ERR_INVALID_ARG
+    assert lib.sd_sparse_decode_sampled(s, fake, fake, fake, fake, fake, N, fake, fake, ws, fake, N) == \
+        sdb.SD_ERR_INVALID_ARG
 
 
 def test_small_workspace_rejected_before_launch(lib):
